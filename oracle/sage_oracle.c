@@ -1,0 +1,454 @@
+/*
+ * sage_oracle.c -- CPU oracle for SageAttention-style quantized attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file: it is used by the test-suite, by the smoke check and by the
+ * CPU-baseline leg of the benchmark.  It shares no code, header, table or
+ * constant generator with the CUDA library.
+ *
+ * It is deliberately plain, slow and single-threaded.  Every function works on
+ * ONE (batch, head) slab; the caller loops over slabs.  Inputs are bf16 bit
+ * patterns (uint16) with an element stride between token rows; channels are
+ * contiguous.
+ *
+ * What it follows (the pages are cited by title and section):
+ *   - "MiniMax H3 接入 SageAttention 实测加速", section 一 (SageAttention 加速了什么):
+ *     Attention(Q,K,V) = Softmax(Q K^T / sqrt(d)) V; SageAttention 2 applies
+ *     low-bit quantization and outlier smoothing to Q K^T; the sm89 kernel
+ *     handles QK in INT8 and PV in FP8.
+ *   - "SDPA稠密注意力模式：大模型推理加速的优化方案", section 三.1 (数学基础):
+ *     the same dense formula with the 1/sqrt(d_k) scale.
+ *   - "GitHub榜单静默期：Attention优化从架构转向推理加速", section 2.2: the
+ *     attention matrix is processed block-wise and never written out; low-bit
+ *     (INT8) representation of chosen attention operands.
+ * Where the pages leave a numeric step open, the reading used here is the one
+ * listed (C1..C9) in the project design notes; each step below names it.
+ *
+ * Two modes:
+ *   oracle_attn_exact  -- the plain definition in fp64 (no smoothing, no
+ *                         quantization).
+ *   oracle_attn_quant  -- the quantization scheme, step by step, in the order
+ *                         smoothing -> block INT8 of Q and K -> integer Q K^T ->
+ *                         dequant -> softmax with an integer-grid (log2) row max
+ *                         -> FP8 e4m3 P and V -> fp64 accumulate -> bf16 output.
+ *                         Steps the GPU performs order-independently in fp32
+ *                         (block amax, scales, codes of Q and V) are emulated
+ *                         here in IEEE fp32 so that they can be compared bit
+ *                         for bit; everything else is fp64.
+ *
+ * Pins (tests that tie this file to something other than itself):
+ *   exact mode      -- brute force on tiny inputs, softmax closed forms
+ *                      (uniform scores, one dominant key, two-key logistic),
+ *                      rows of weights summing to one, uniform V returning V,
+ *                      invariance under a per-channel K offset.
+ *   quant mode      -- with every error source switched off it must equal the
+ *                      exact mode; the e4m3 and bf16 rounding helpers against
+ *                      the format definitions and a library cast; the int8
+ *                      block codes against closed forms; the one-pass
+ *                      integer-grid softmax against a tile-by-tile replay of
+ *                      the online algorithm.
+ *
+ * Build:  gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
+ *             -fexcess-precision=standard -o liboracle.so sage_oracle.c -lm
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <fenv.h>
+
+#define ORACLE_Q_BLOCK 128 /* Q tokens per quantization block (reading C3) */
+#define ORACLE_K_BLOCK 64  /* K tokens per quantization block (reading C3) */
+#define ORACLE_E4M3_MAX 448.0
+
+/* ------------------------------------------------------------------------ */
+/* Number formats                                                           */
+/* ------------------------------------------------------------------------ */
+
+/* bf16 bit pattern -> value: the top 16 bits of an IEEE binary32. Exact. */
+double oracle_bf16_to_double(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+static float bf16_to_float(uint16_t h)
+{
+    uint32_t u = ((uint32_t)h) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a double to bf16, nearest-even (1 sign, 8 exponent, 7 fraction bits),
+ * returned as the bit pattern.  The rounding is done once, directly on the
+ * double, at the spacing of the target binade (no detour through binary32). */
+uint16_t oracle_bf16_rne(double x)
+{
+    if (isnan(x)) return 0x7fc0;
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    double a = fabs(x);
+    if (a == 0.0) return sign;
+    if (isinf(a)) return sign | 0x7f80;
+    int e;
+    frexp(a, &e);             /* a = f * 2^e with f in [0.5, 1) */
+    /* bf16 keeps 8 significant bits; normals start at 2^-126. */
+    int exp_unbiased = e - 1; /* a in [2^exp_unbiased, 2^(exp_unbiased+1)) */
+    double q;                 /* significand in units of the last place */
+    int lsb_exp;
+    if (exp_unbiased < -126) lsb_exp = -126 - 7; /* subnormal spacing 2^-133 */
+    else lsb_exp = exp_unbiased - 7;
+    q = ldexp(a, -lsb_exp); /* exact: scaling by a power of two */
+    double r = nearbyint(q); /* ties to even in the default rounding mode */
+    double v = ldexp(r, lsb_exp);
+    if (v > 0x1.fep127) return sign | 0x7f80; /* rounds past the largest finite -> inf */
+    float vf = (float)v; /* exact: v has at most 8 significant bits */
+    uint32_t u;
+    memcpy(&u, &vf, sizeof u);
+    return (uint16_t)(sign | ((u >> 16) & 0x7fff));
+}
+
+/* e4m3 ("fn" variant: no infinities, one NaN pattern S.1111.111).
+ * Value of a code: exponent field E (4 bits, bias 7), mantissa M (3 bits);
+ * E > 0: 2^(E-7) * (1 + M/8); E == 0: 2^-6 * (M/8).  Largest finite 448. */
+double oracle_e4m3_decode(uint8_t code)
+{
+    int s = code >> 7, E = (code >> 3) & 0xf, M = code & 7;
+    double v;
+    if (E == 0xf && M == 7) return NAN;
+    if (E == 0) v = ldexp((double)M / 8.0, -6);
+    else v = ldexp(1.0 + (double)M / 8.0, E - 7);
+    return s ? -v : v;
+}
+
+/* Round a finite double to e4m3, nearest-even, saturating to +-448
+ * ("satfinite").  Returns the code. */
+uint8_t oracle_e4m3_encode(double x)
+{
+    uint8_t s = signbit(x) ? 0x80 : 0;
+    double a = fabs(x);
+    if (isnan(x)) return 0x7f;
+    if (a >= ORACLE_E4M3_MAX) return s | 0x7e; /* 448 = E 15, M 6 */
+    if (a == 0.0) return s;
+    int e;
+    frexp(a, &e);
+    int exp_unbiased = e - 1;   /* a in [2^exp, 2^(exp+1)) */
+    int lsb_exp;
+    if (exp_unbiased < -6) lsb_exp = -9; /* subnormal spacing 2^-9 */
+    else lsb_exp = exp_unbiased - 3;
+    double r = nearbyint(ldexp(a, -lsb_exp)); /* ties to even */
+    double v = ldexp(r, lsb_exp);
+    if (v > ORACLE_E4M3_MAX) v = ORACLE_E4M3_MAX; /* cannot happen below 448 */
+    /* encode v exactly */
+    if (v == 0.0) return s;
+    int ev;
+    frexp(v, &ev);
+    int E = (ev - 1) + 7;
+    uint8_t code;
+    if (E <= 0) { /* subnormal: v = M * 2^-9 */
+        code = (uint8_t)(int)ldexp(v, 9);
+    } else {
+        double frac = ldexp(v, -(ev - 1)) - 1.0; /* in [0,1) */
+        int M = (int)(frac * 8.0);
+        code = (uint8_t)((E << 3) | M);
+    }
+    return s | code;
+}
+
+double oracle_e4m3_round(double x) { return oracle_e4m3_decode(oracle_e4m3_encode(x)); }
+
+/* ------------------------------------------------------------------------ */
+/* Exact mode: the plain definition (dense formula of both pages)           */
+/* ------------------------------------------------------------------------ */
+
+/* out[r][c] = sum_j w_rj v_j[c],  w_rj = exp(s_rj - max_j s) / sum_j exp(...),
+ * s_rj = sm_scale * sum_c q_r[c] k_j[c].  All fp64; inputs decoded exactly.
+ * If weights != NULL, the softmax weights of each requested row are written
+ * there ([nrows][N]). */
+int oracle_attn_exact(const uint16_t *q, int64_t q_rs,
+                      const uint16_t *k, int64_t k_rs,
+                      const uint16_t *v, int64_t v_rs,
+                      int N, int d, double sm_scale,
+                      const int32_t *rows, int nrows,
+                      double *out, double *weights)
+{
+    if (N <= 0 || d <= 0) return -1;
+    double *s = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!s) return -2;
+    for (int ri = 0; ri < nrows; ++ri) {
+        int r = rows[ri];
+        if (r < 0 || r >= N) { free(s); return -3; }
+        double smax = -INFINITY;
+        for (int j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c)
+                acc += oracle_bf16_to_double(q[(int64_t)r * q_rs + c]) *
+                       oracle_bf16_to_double(k[(int64_t)j * k_rs + c]);
+            s[j] = acc * sm_scale;
+            if (s[j] > smax) smax = s[j];
+        }
+        double l = 0.0;
+        for (int j = 0; j < N; ++j) { s[j] = exp(s[j] - smax); l += s[j]; }
+        for (int c = 0; c < d; ++c) out[(int64_t)ri * d + c] = 0.0;
+        for (int j = 0; j < N; ++j) {
+            double w = s[j] / l;
+            if (weights) weights[(int64_t)ri * N + j] = w;
+            for (int c = 0; c < d; ++c)
+                out[(int64_t)ri * d + c] += w * oracle_bf16_to_double(v[(int64_t)j * v_rs + c]);
+        }
+    }
+    free(s);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantization (smoothing, block INT8 for Q and K, per-channel e4m3 for V)  */
+/* ------------------------------------------------------------------------ */
+
+/* Symmetric INT8 code of one fp32 value given the fp32 reciprocal scale:
+ * round half to even of the fp32 product, clamped to [-127, 127] (reading C2). */
+static int8_t int8_code(float x, float inv)
+{
+    float y = x * inv;           /* one IEEE fp32 multiply */
+    float r = nearbyintf(y);     /* ties to even */
+    if (r > 127.0f) r = 127.0f;
+    if (r < -127.0f) r = -127.0f;
+    return (int8_t)r;
+}
+
+/*
+ * Quantize one (b,h) slab (all N tokens).
+ *   k_mean[c]  = mean over the N tokens of K[:,c]            (reading C1; fp64,
+ *                stored rounded to fp32)
+ *   Q block b (128 tokens, reading C3):  amax = max |Q| over the block's valid
+ *                tokens and all channels; q_scale = fp32(amax/127);
+ *                code = rne(fp32(Q * fp32(127/amax)))          (reading C2)
+ *   K block b (64 tokens): the same on fp32(K - k_mean32)     (readings C1-C3)
+ *   V channel c: amax = max_n |V[n,c]|; v_scale = fp32(amax/448);
+ *                code = e4m3_rn_satfinite(fp32(V * fp32(448/amax)))  (reading C7)
+ * A zero amax gives scale 0 and all-zero codes.
+ * smooth_k = 0 skips the mean subtraction (used by tests).
+ * Output layouts (row-major, token-major, no padding):
+ *   q_i8[N][d], q_scale[ceil(N/128)], k_i8[N][d], k_scale[ceil(N/64)],
+ *   k_mean[d], v_e4m3[N][d], v_scale[d].
+ */
+int oracle_quantize(const uint16_t *q, int64_t q_rs,
+                    const uint16_t *k, int64_t k_rs,
+                    const uint16_t *v, int64_t v_rs,
+                    int N, int d, int smooth_k,
+                    int8_t *q_i8, float *q_scale,
+                    int8_t *k_i8, float *k_scale, float *k_mean,
+                    uint8_t *v_e4m3, float *v_scale)
+{
+    if (N <= 0 || d <= 0) return -1;
+    /* smoothing statistic */
+    for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int n = 0; n < N; ++n) acc += oracle_bf16_to_double(k[(int64_t)n * k_rs + c]);
+        k_mean[c] = smooth_k ? (float)(acc / (double)N) : 0.0f;
+    }
+    /* Q blocks */
+    int nqb = (N + ORACLE_Q_BLOCK - 1) / ORACLE_Q_BLOCK;
+    for (int b = 0; b < nqb; ++b) {
+        int n0 = b * ORACLE_Q_BLOCK, n1 = n0 + ORACLE_Q_BLOCK;
+        if (n1 > N) n1 = N;
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float a = fabsf(bf16_to_float(q[(int64_t)n * q_rs + c]));
+                if (a > amax) amax = a;
+            }
+        float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+        q_scale[b] = amax > 0.0f ? amax / 127.0f : 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c)
+                q_i8[(int64_t)n * d + c] =
+                    amax > 0.0f ? int8_code(bf16_to_float(q[(int64_t)n * q_rs + c]), inv) : 0;
+    }
+    /* K blocks on the smoothed keys */
+    int nkb = (N + ORACLE_K_BLOCK - 1) / ORACLE_K_BLOCK;
+    for (int b = 0; b < nkb; ++b) {
+        int n0 = b * ORACLE_K_BLOCK, n1 = n0 + ORACLE_K_BLOCK;
+        if (n1 > N) n1 = N;
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float ks = bf16_to_float(k[(int64_t)n * k_rs + c]) - k_mean[c];
+                float a = fabsf(ks);
+                if (a > amax) amax = a;
+            }
+        float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+        k_scale[b] = amax > 0.0f ? amax / 127.0f : 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float ks = bf16_to_float(k[(int64_t)n * k_rs + c]) - k_mean[c];
+                k_i8[(int64_t)n * d + c] = amax > 0.0f ? int8_code(ks, inv) : 0;
+            }
+    }
+    /* V per channel */
+    for (int c = 0; c < d; ++c) {
+        float amax = 0.0f;
+        for (int n = 0; n < N; ++n) {
+            float a = fabsf(bf16_to_float(v[(int64_t)n * v_rs + c]));
+            if (a > amax) amax = a;
+        }
+        float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+        v_scale[c] = amax > 0.0f ? amax / 448.0f : 0.0f;
+        for (int n = 0; n < N; ++n) {
+            float x = bf16_to_float(v[(int64_t)n * v_rs + c]) * inv;
+            v_e4m3[(int64_t)n * d + c] = amax > 0.0f ? oracle_e4m3_encode((double)x) : 0;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quant-emulation attention                                                */
+/* ------------------------------------------------------------------------ */
+
+/* Switches for the error sources (all 1 = the scheme as specified). */
+typedef struct {
+    int int8_qk;    /* 0: scores from the exact smoothed product q.(k-mean)   */
+    int fp8_p;      /* 0: P kept unrounded                                     */
+    int fp8_v;      /* 0: V kept exact (no e4m3, no scale)                      */
+    int round_bf16; /* 0: out_bf16 still written, but from the unrounded value */
+    int smooth_k;   /* 0: no mean subtraction before K quantization            */
+} oracle_quant_flags;
+
+/*
+ * For each requested query row r of one slab:
+ *   S_rj   = sum_c qcode[r,c] * kcode[j,c]                 (exact integer)
+ *   c_rj   = fp32( fp32(q_scale[r/128] * s_l2) * k_scale[j/64] ),
+ *            s_l2 = fp32(fp32(sm_scale) * fp32(log2 e))    (reading C4)
+ *   x_rj   = S_rj * c_rj                                   (fp64; log2 units)
+ *   m_r    = ceil(max_j x_rj)                              (reading C5)
+ *   p_rj   = 2^(x_rj - m_r)            l_r = sum_j p_rj   (fp64, unrounded)
+ *   P_rj   = e4m3_rn_satfinite(448 p_rj)                   (reading C6)
+ *   O_rc   = sum_j P_rj * vcode_value[j,c]                 (fp64)
+ *   out_rc = bf16_rne( O_rc * v_scale[c] / (448 l_r) )    (reading C8)
+ * The dropped smoothing term q.mean is a per-row constant of the scores and
+ * cancels in the softmax (reading C1).  Because m_r lies on the integer grid,
+ * a tiled online evaluation that rescales by 2^(m_old - m_new) produces the
+ * same P codes as this one-pass form wherever 448 p stays in e4m3's normal
+ * range (reading C5); below it (448 p < 2^-6) the one-pass form is used.
+ * out_f64 (may be NULL) receives the value before the bf16 rounding,
+ * out_bf16 (may be NULL) the rounded bit pattern; both [nrows][d].
+ */
+int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
+                      const uint16_t *k, int64_t k_rs,
+                      const uint16_t *v, int64_t v_rs,
+                      int N, int d, float sm_scale,
+                      const oracle_quant_flags *flags,
+                      const int32_t *rows, int nrows,
+                      double *out_f64, uint16_t *out_bf16)
+{
+    if (N <= 0 || d <= 0 || !flags) return -1;
+    int nqb = (N + ORACLE_Q_BLOCK - 1) / ORACLE_Q_BLOCK;
+    int nkb = (N + ORACLE_K_BLOCK - 1) / ORACLE_K_BLOCK;
+    size_t nd = (size_t)N * (size_t)d;
+    int8_t *qc = (int8_t *)malloc(nd), *kc = (int8_t *)malloc(nd);
+    uint8_t *vc = (uint8_t *)malloc(nd);
+    float *qs = (float *)malloc(sizeof(float) * nqb), *ks = (float *)malloc(sizeof(float) * nkb);
+    float *km = (float *)malloc(sizeof(float) * d), *vs = (float *)malloc(sizeof(float) * d);
+    double *x = (double *)malloc(sizeof(double) * (size_t)N);
+    double *vval = (double *)malloc(sizeof(double) * nd);
+    double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    int rc = 0;
+    if (!qc || !kc || !vc || !qs || !ks || !km || !vs || !x || !vval || !o) { rc = -2; goto done; }
+
+    rc = oracle_quantize(q, q_rs, k, k_rs, v, v_rs, N, d, flags->smooth_k,
+                         qc, qs, kc, ks, km, vc, vs);
+    if (rc) goto done;
+
+    /* value of V used in the P.V product, already multiplied by its scale */
+    for (int n = 0; n < N; ++n)
+        for (int c = 0; c < d; ++c)
+            vval[(size_t)n * d + c] =
+                flags->fp8_v ? oracle_e4m3_decode(vc[(size_t)n * d + c]) * (double)vs[c]
+                             : oracle_bf16_to_double(v[(int64_t)n * v_rs + c]);
+
+    const float log2e_f = (float)1.4426950408889634; /* log2(e) rounded to fp32 */
+    const float s_l2 = sm_scale * log2e_f;           /* one fp32 multiply */
+
+    for (int ri = 0; ri < nrows; ++ri) {
+        int r = rows[ri];
+        if (r < 0 || r >= N) { rc = -3; goto done; }
+        float sq = qs[r / ORACLE_Q_BLOCK];
+        float cq = sq * s_l2; /* fp32 */
+        double xmax = -INFINITY;
+        for (int j = 0; j < N; ++j) {
+            if (flags->int8_qk) {
+                int64_t S = 0;
+                for (int c = 0; c < d; ++c)
+                    S += (int64_t)qc[(size_t)r * d + c] * (int64_t)kc[(size_t)j * d + c];
+                float cj = cq * ks[j / ORACLE_K_BLOCK]; /* fp32 */
+                x[j] = (double)S * (double)cj;
+            } else {
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc += oracle_bf16_to_double(q[(int64_t)r * q_rs + c]) *
+                           (oracle_bf16_to_double(k[(int64_t)j * k_rs + c]) -
+                            (flags->smooth_k ? (double)km[c] : 0.0));
+                x[j] = acc * (double)sm_scale * 1.4426950408889634;
+            }
+            if (x[j] > xmax) xmax = x[j];
+        }
+        double m = ceil(xmax);
+        double l = 0.0;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        for (int j = 0; j < N; ++j) {
+            double p = exp2(x[j] - m);
+            l += p;
+            double P = flags->fp8_p ? oracle_e4m3_round(p * ORACLE_E4M3_MAX) : p * ORACLE_E4M3_MAX;
+            if (P == 0.0) continue;
+            for (int c = 0; c < d; ++c) o[c] += P * vval[(size_t)j * d + c];
+        }
+        for (int c = 0; c < d; ++c) {
+            double y = o[c] / (ORACLE_E4M3_MAX * l);
+            if (out_f64) out_f64[(size_t)ri * d + c] = y;
+            if (out_bf16) out_bf16[(size_t)ri * d + c] = oracle_bf16_rne(y);
+        }
+    }
+done:
+    free(qc); free(kc); free(vc); free(qs); free(ks); free(km); free(vs);
+    free(x); free(vval); free(o);
+    return rc;
+}
+
+/* Integer score tile from given codes: s[i][j] = sum_c a[i][c] * b[j][c]
+ * for i < m, j < n (row-major codes with row strides a_rs, b_rs).  This is
+ * the definition of the INT8 product with int32 accumulation; |s| <= d*127^2
+ * fits int32 for d <= 133000. */
+int oracle_int8_gemm_nt(const int8_t *a, int64_t a_rs, const int8_t *b, int64_t b_rs,
+                        int m, int n, int d, int32_t *s)
+{
+    for (int i = 0; i < m; ++i)
+        for (int j = 0; j < n; ++j) {
+            int64_t acc = 0;
+            for (int c = 0; c < d; ++c)
+                acc += (int64_t)a[(int64_t)i * a_rs + c] * (int64_t)b[(int64_t)j * b_rs + c];
+            s[(int64_t)i * n + j] = (int32_t)acc;
+        }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Array forms of the format helpers (for the tests)                        */
+/* ------------------------------------------------------------------------ */
+
+void oracle_e4m3_encode_array(const double *x, int64_t n, uint8_t *code)
+{
+    for (int64_t i = 0; i < n; ++i) code[i] = oracle_e4m3_encode(x[i]);
+}
+
+void oracle_e4m3_decode_array(const uint8_t *code, int64_t n, double *x)
+{
+    for (int64_t i = 0; i < n; ++i) x[i] = oracle_e4m3_decode(code[i]);
+}
+
+void oracle_bf16_rne_array(const double *x, int64_t n, uint16_t *h)
+{
+    for (int64_t i = 0; i < n; ++i) h[i] = oracle_bf16_rne(x[i]);
+}
