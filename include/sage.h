@@ -1,0 +1,187 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) quantized-attention library (libsage.so).
+ *
+ * The library computes the forward pass of SageAttention-style quantized
+ * attention:  out = softmax(Q K^T * sm_scale) V  with
+ *   - K smoothed by subtracting its per-(batch, head, channel) mean over tokens,
+ *   - Q in INT8 per 128-token block and K in INT8 per 64-token block
+ *     (symmetric, one fp32 scale per block),
+ *   - S = Q K^T on the INT8 tensor cores with int32 accumulation, dequantized
+ *     by the block scales,
+ *   - an online softmax in base 2 whose running row max stays on the integer
+ *     grid (rescale factors are exact powers of two),
+ *   - P (scaled by 448) and V (per-channel scale) in FP8 e4m3, P V on the FP8
+ *     tensor cores with fp32 accumulation, bf16 output.
+ *
+ * Sources (web pages, by title and section):
+ *   [H3]   "MiniMax H3 接入 SageAttention 实测加速", section 一 "SageAttention 加速了什么":
+ *          Attention(Q,K,V) = Softmax(Q K^T / sqrt(d)) V; low-bit quantization and
+ *          outlier smoothing of Q K^T; INT8 for QK and FP8 for PV.
+ *   [SDPA] "SDPA稠密注意力模式：大模型推理加速的优化方案", section 三.1 "数学基础":
+ *          the dense formula with the 1/sqrt(d_k) scale (the dense reference).
+ *   [BLOG] "GitHub榜单静默期：Attention优化从架构转向推理加速", section 2.2:
+ *          block-wise computation that never writes the attention matrix out.
+ *   [SOL]  "ComfyUI-sol-attn" page, "核心亮点" items 2 and 4: zero-copy reads of a
+ *          fused-qkv strided view; explicit, logged rejection of unsupported
+ *          inputs instead of a silent fallback.
+ * Numeric points the pages leave open follow the readings C1..C9 of the
+ * project's design notes (block sizes, rounding modes, integer-grid row max,
+ * 448 P scale, per-channel V scale, fp32 accumulation, bf16 RNE output).
+ *
+ * Conventions for every entry point
+ *   - Tensors are described by a base pointer plus four int64 ELEMENT strides in
+ *     (b, h, n, c) order; the channel stride must be 1.  A fused [B,N,3,H,d]
+ *     qkv buffer is passed as three views with strides (N*3*H*d, d, 3*H*d, 1)
+ *     and read in place (no copy).
+ *   - Inputs and output are bf16.  d must be 64 or 128; N >= 1; B, H >= 1.
+ *     Base pointers must be 16-byte aligned and the b, h, n strides multiples
+ *     of 8 elements (16-byte vectors).  Otherwise SAGE_ERR_INVALID_ARG (bad
+ *     pointer/stride/shape/scale) or SAGE_ERR_UNSUPPORTED (d, dtype) is
+ *     returned before anything is launched.
+ *   - N_pad = ceil(N/128)*128.  Padded rows of every code buffer are written
+ *     as zeros; padded blocks get scale 0.
+ *   - Every device buffer is owned by the caller; the library keeps no pointer
+ *     after a call returns.  Calls are asynchronous on `stream` and return
+ *     after the launches.  A kernel that gives up waiting on an internal
+ *     barrier (a bounded wait) records it in a device error word that
+ *     sage_check() reports as SAGE_ERR_TIMEOUT.
+ *   - There is no fallback of any kind: an unsupported input is an error.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t (the runtime's opaque stream pointer). */
+typedef struct CUstream_st *sage_stream_t;
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad stride, shape or scale   */
+    SAGE_ERR_UNSUPPORTED = 2,  /* head dim not in {64,128}                             */
+    SAGE_ERR_WORKSPACE = 3,    /* workspace given but smaller than required             */
+    SAGE_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed (message has it)    */
+    SAGE_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (see sage_check)   */
+} sage_status_t;
+
+/* Human-readable name of a status code (static string). */
+const char *sage_status_string(sage_status_t status);
+
+/* Detail of the last error raised on the calling host thread ("" if none). */
+const char *sage_last_error_message(void);
+
+/* Synchronize `stream`, then read and clear the device error word.  Returns
+ * SAGE_ERR_TIMEOUT if any kernel of this library gave up on a bounded wait
+ * since the last check, SAGE_ERR_CUDA on a failed synchronize, else SAGE_OK. */
+sage_status_t sage_check(sage_stream_t stream);
+
+/* Bytes of scratch sage_attn_fwd needs for this shape (codes, scales, stats).
+ * 0 for an invalid shape.  Layout inside it is private. */
+size_t sage_attn_workspace_bytes(int B, int H, int N, int d);
+
+/* Bytes of scratch sage_quant_qk / sage_quant_v need (the per-chunk partial
+ * statistics of the smoothing mean and of the V channel maxima). */
+size_t sage_quant_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * sage_quant_qk -- smoothing plus block quantization of Q and K ([H3] section 一;
+ * readings C1-C3).
+ *   k_mean[b,h,c] = (1/N) sum_n K[b,h,n,c]                 (fp32 accumulation)
+ *   Q, per 128-token block:  amax = max|Q| over the block's valid tokens and all
+ *       channels; q_scale = amax/127; q_i8 = rne(Q * (127/amax)) in [-127,127]
+ *   K, the same per 64-token block on (K - k_mean).
+ * Outputs (device, caller-allocated, contiguous):
+ *   q_i8    int8  [B,H,N_pad,d]      q_scale float [B,H,N_pad/128]
+ *   k_i8    int8  [B,H,N_pad,d]      k_scale float [B,H,N_pad/64]
+ *   k_mean  float [B,H,d]  (may be NULL)
+ * workspace: >= sage_quant_workspace_bytes() device bytes, or NULL to let the
+ * library take it from the stream-ordered allocator for the duration of the call.
+ */
+sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4],
+                            const void *k_bf16, const int64_t k_stride[4],
+                            int B, int H, int N, int d,
+                            int8_t *q_i8, float *q_scale,
+                            int8_t *k_i8, float *k_scale, float *k_mean,
+                            void *workspace, size_t workspace_bytes,
+                            sage_stream_t stream);
+
+/*
+ * sage_quant_v -- V to FP8 e4m3 with one scale per (b,h,channel) ([H3] "FP8 for
+ * PV"; reading C7):  amax_c = max_n |V|;  v_scale = amax_c/448;
+ * v_t8[b,h,c,n] = e4m3_rn_satfinite(V * (448/amax_c)).
+ * Outputs: v_t8 uint8 (e4m3 bits) [B,H,d,N_pad] -- channel-major, i.e. V
+ * transposed so that the P.V operand is K-major; v_scale float [B,H,d].
+ * workspace as for sage_quant_qk.
+ */
+sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4],
+                           int B, int H, int N, int d,
+                           uint8_t *v_t8, float *v_scale,
+                           void *workspace, size_t workspace_bytes,
+                           sage_stream_t stream);
+
+/*
+ * sage_attn_quantized -- the fused attention kernel alone, on codes produced by
+ * sage_quant_qk / sage_quant_v (or any producer of the same layouts):
+ *   x = S_int * (q_scale * sm_scale * log2(e) * k_scale)   (int32 S on tcgen05 kind::i8)
+ *   running max m on the integer grid; p = 2^(x - m); l = sum p (fp32)
+ *   P = e4m3(448 p) in tensor memory; O += P V on tcgen05 kind::f8f6f4 (fp32)
+ *   out = O * v_scale / (448 l) -> bf16 (round to nearest even)
+ * [BLOG] section 2.2 (block-wise, no N x N matrix); readings C4-C8.
+ * out: bf16, strides as described above.  sm_scale finite and > 0.
+ */
+sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale,
+                                  const int8_t *k_i8, const float *k_scale,
+                                  const uint8_t *v_t8, const float *v_scale,
+                                  void *out, const int64_t o_stride[4],
+                                  int B, int H, int N, int d, float sm_scale,
+                                  sage_stream_t stream);
+
+/*
+ * sage_attn_fwd -- the whole quantized attention forward: sage_quant_qk,
+ * sage_quant_v and sage_attn_quantized on scratch taken from `workspace`
+ * (>= sage_attn_workspace_bytes(B,H,N,d) bytes, or NULL: stream-ordered
+ * allocation for the duration of the call).  q, k, v may be strided views of
+ * one fused qkv buffer ([SOL] item 2).  sm_scale is usually 1/sqrt(d).
+ */
+sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4],
+                            const void *k, const int64_t k_stride[4],
+                            const void *v, const int64_t v_stride[4],
+                            void *out, const int64_t o_stride[4],
+                            int B, int H, int N, int d, float sm_scale,
+                            void *workspace, size_t workspace_bytes,
+                            sage_stream_t stream);
+
+/*
+ * sage_attn_dense_ref_gpu -- plain dense attention on the CUDA cores in fp32
+ * ([SDPA] section 三.1, [H3] section 一): no quantization, no tensor cores,
+ * exact softmax with a running max (fp32 expf).  For A/B checks only.
+ */
+sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4],
+                                      const void *k, const int64_t k_stride[4],
+                                      const void *v, const int64_t v_stride[4],
+                                      void *out, const int64_t o_stride[4],
+                                      int B, int H, int N, int d, float sm_scale,
+                                      sage_stream_t stream);
+
+/*
+ * sage_debug_qk_tile -- export one int32 S tile (128 queries x 128 keys) of
+ * slab (b,h): rows q_tile*128.., keys kv_tile*128.., computed by the same
+ * TMA + tcgen05 kind::i8 path the attention kernel uses.  q_i8/k_i8 as
+ * written by sage_quant_qk.  s_out: device int32 [128][128], row-major.
+ * Entries for keys or queries beyond N_pad are what the zero padding gives (0).
+ */
+sage_status_t sage_debug_qk_tile(const int8_t *q_i8, const int8_t *k_i8,
+                                 int B, int H, int N, int d,
+                                 int b, int h, int q_tile, int kv_tile,
+                                 int32_t *s_out, sage_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H_ */

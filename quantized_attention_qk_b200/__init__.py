@@ -1,0 +1,218 @@
+"""quantized_attention_qk_b200 -- SageAttention-style quantized attention on B200.
+
+Thin Python binding of ``lib/libsage.so`` (include/sage.h).  Every function
+here only marshals torch tensors into pointers, strides and sizes and calls the
+C ABI function of the same name; all arithmetic runs in the library's CUDA
+kernels.  torch provides device memory and streams.  There is no fallback: if
+the library is missing or a call fails, an exception is raised.
+
+Tensors are [B, H, N, d] bf16 views with channel stride 1 (e.g. slices of a
+fused [B, N, 3, H, d] qkv buffer, read in place).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+__all__ = [
+    "SageError", "lib", "sage_attn_fwd", "sage_attn_quantized", "sage_quant_qk", "sage_quant_v",
+    "sage_attn_dense_ref_gpu", "sage_debug_qk_tile", "sage_attn_workspace_bytes",
+    "sage_quant_workspace_bytes", "sage_check", "sage_attn_fwd_host", "n_pad",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libsage.so")
+Q_BLOCK, K_BLOCK = 128, 64
+
+SAGE_STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED", 3: "SAGE_ERR_WORKSPACE",
+               4: "SAGE_ERR_CUDA", 5: "SAGE_ERR_TIMEOUT"}
+
+
+class SageError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{SAGE_STATUS.get(status, status)}: {message}")
+        self.status = status
+
+
+_lib = None
+_P, _I64P, _I32, _SZ = ctypes.c_void_p, ctypes.POINTER(ctypes.c_int64), ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "sage_status_string": ([_I32], ctypes.c_char_p),
+    "sage_last_error_message": ([], ctypes.c_char_p),
+    "sage_check": ([_P], _I32),
+    "sage_attn_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_quant_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_quant_qk": ([_P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
+    "sage_quant_v": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
+    "sage_attn_quantized": ([_P, _P, _P, _P, _P, _P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float, _P], _I32),
+    "sage_attn_fwd": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                       _P, _SZ, _P], _I32),
+    "sage_attn_dense_ref_gpu": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32,
+                                 ctypes.c_float, _P], _I32),
+    "sage_debug_qk_tile": ([_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
+}
+
+
+def lib():
+    """Load libsage.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with quantized_attention_qk_b200.build.build()")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def _raise(status: int):
+    if status != 0:
+        raise SageError(status, lib().sage_last_error_message().decode(errors="replace"))
+
+
+def _strides(t: torch.Tensor):
+    return (ctypes.c_int64 * 4)(*t.stride())
+
+
+def _stream(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def n_pad(N: int) -> int:
+    return -(-N // Q_BLOCK) * Q_BLOCK
+
+
+def _check_qkv(*ts):
+    for t in ts:
+        if t.dim() != 4 or t.dtype != torch.bfloat16 or not t.is_cuda:
+            raise ValueError("expected bf16 CUDA tensors of shape [B, H, N, d]")
+
+
+def sage_attn_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().sage_attn_workspace_bytes(B, H, N, d))
+
+
+def sage_quant_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().sage_quant_workspace_bytes(B, H, N, d))
+
+
+def sage_check(stream=None, device=None):
+    _raise(lib().sage_check(_stream(stream, device)))
+
+
+def sage_quant_qk(q, k, workspace=None, stream=None):
+    """Smoothing + block INT8 quantization.  Returns dict of device tensors:
+    q_i8 [B,H,N_pad,d] int8, q_scale [B,H,N_pad/128], k_i8, k_scale [B,H,N_pad/64], k_mean [B,H,d]."""
+    _check_qkv(q, k)
+    B, H, N, d = q.shape
+    dev = q.device
+    npd = n_pad(N)
+    r = dict(q_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
+             q_scale=torch.empty(B, H, npd // Q_BLOCK, dtype=torch.float32, device=dev),
+             k_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
+             k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
+             k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _raise(lib().sage_quant_qk(_ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
+                               _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]), _ptr(r["k_scale"]),
+                               _ptr(r["k_mean"]), _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    return r
+
+
+def sage_quant_v(v, workspace=None, stream=None):
+    """V -> e4m3 with per-channel scales.  Returns (v_t8 uint8 [B,H,d,N_pad], v_scale [B,H,d])."""
+    _check_qkv(v)
+    B, H, N, d = v.shape
+    dev = v.device
+    v_t8 = torch.empty(B, H, d, n_pad(N), dtype=torch.uint8, device=dev)
+    v_scale = torch.empty(B, H, d, dtype=torch.float32, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _raise(lib().sage_quant_v(_ptr(v), _strides(v), B, H, N, d, _ptr(v_t8), _ptr(v_scale), _ptr(workspace),
+                              ws_bytes, _stream(stream, dev)))
+    return v_t8, v_scale
+
+
+def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_t8, v_scale, N: int, sm_scale=None, out=None, stream=None):
+    """The fused attention kernel on existing codes; returns bf16 [B,H,N,d]."""
+    B, H, _, d = q_i8.shape
+    dev = q_i8.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    for t in (q_i8, q_scale, k_i8, k_scale, v_t8, v_scale):
+        if not t.is_contiguous():
+            raise ValueError("code and scale tensors must be contiguous")
+    _raise(lib().sage_attn_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_t8),
+                                     _ptr(v_scale), _ptr(out), _strides(out), B, H, N, d,
+                                     ctypes.c_float(sm_scale), _stream(stream, dev)))
+    return out
+
+
+def sage_attn_fwd(q, k, v, sm_scale=None, out=None, workspace=None, stream=None):
+    """Quantized attention forward on device tensors; returns bf16 [B,H,N,d]."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    dev = q.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _raise(lib().sage_attn_fwd(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                               _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                               _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    return out
+
+
+def sage_attn_dense_ref_gpu(q, k, v, sm_scale=None, out=None, stream=None):
+    """Dense fp32 CUDA-core attention (A/B reference); returns bf16 [B,H,N,d]."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=q.device)
+    _raise(lib().sage_attn_dense_ref_gpu(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                         _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                         _stream(stream, q.device)))
+    return out
+
+
+def sage_debug_qk_tile(q_i8, k_i8, N: int, b: int, h: int, q_tile: int, kv_tile: int, stream=None):
+    """int32 [128,128] S tile of slab (b,h) computed on the tcgen05 INT8 path."""
+    B, H, _, d = q_i8.shape
+    s = torch.empty(128, 128, dtype=torch.int32, device=q_i8.device)
+    _raise(lib().sage_debug_qk_tile(_ptr(q_i8), _ptr(k_i8), B, H, N, d, b, h, q_tile, kv_tile, _ptr(s),
+                                    _stream(stream, q_i8.device)))
+    return s
+
+
+def sage_attn_fwd_host(qkv_host, B, H, N, d, layout="fused", sm_scale=None, device="cuda", out_host=None,
+                       workspace=None, stream=None):
+    """End-to-end call on HOST memory: copy the (pinned) input to the device,
+    run sage_attn_fwd, copy the bf16 result back into ``out_host``.
+
+    ``qkv_host`` is one pinned bf16 buffer: [B,N,3,H,d] for layout "fused",
+    [3,B,H,N,d] for "contiguous".  Returns ``out_host`` ([B,H,N,d], pinned)."""
+    dev_buf = qkv_host.to(device, non_blocking=True)
+    if layout == "fused":
+        q, k, v = (dev_buf[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    else:
+        q, k, v = dev_buf[0], dev_buf[1], dev_buf[2]
+    out = sage_attn_fwd(q, k, v, sm_scale=sm_scale, workspace=workspace, stream=stream)
+    if out_host is None:
+        out_host = torch.empty(B, H, N, d, dtype=torch.bfloat16, pin_memory=True)
+    out_host.copy_(out, non_blocking=True)
+    return out_host

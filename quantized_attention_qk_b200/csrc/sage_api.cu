@@ -1,0 +1,311 @@
+// sage_api.cu -- the extern "C" entry points declared in include/sage.h:
+// argument validation (before any launch), scratch sizing and carving,
+// stream-ordered launches, status codes and the per-thread error message.
+// Unsupported inputs are rejected with an explicit status, never routed
+// elsewhere (the "strict" behaviour the ComfyUI-sol-attn page describes in
+// its 核心亮点 item 4).
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "sage.h"
+#include "sage_internal.h"
+
+namespace sage {
+namespace {
+
+thread_local std::string g_last_error;
+
+sage_status_t fail(sage_status_t st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+sage_status_t cuda_fail(cudaError_t e, const char *what) {
+    return fail(SAGE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr size_t kAlign = 1024;
+size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+sage_status_t check_shape(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1) return fail(SAGE_ERR_INVALID_ARG, "shape B=%d H=%d N=%d must be positive", B, H, N);
+    if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d=%d is not supported (64 or 128)", d);
+    if ((int64_t)B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
+    if (N > (1 << 24)) return fail(SAGE_ERR_UNSUPPORTED, "N=%d exceeds 2^24 tokens", N);
+    return SAGE_OK;
+}
+
+// bf16 tensor view: 16-byte aligned base, channel stride 1, other strides
+// multiples of 8 elements (so every row starts on a 16-byte boundary).
+sage_status_t check_view(const void *p, const int64_t *st, const char *name) {
+    if (!p) return fail(SAGE_ERR_INVALID_ARG, "%s is null", name);
+    if (!st) return fail(SAGE_ERR_INVALID_ARG, "%s strides are null", name);
+    if (reinterpret_cast<uintptr_t>(p) % 16) return fail(SAGE_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    if (st[3] != 1) return fail(SAGE_ERR_INVALID_ARG, "%s channel stride is %lld, must be 1", name, (long long)st[3]);
+    for (int i = 0; i < 3; ++i)
+        if (st[i] % 8 != 0)
+            return fail(SAGE_ERR_INVALID_ARG, "%s stride[%d]=%lld is not a multiple of 8 elements", name, i,
+                        (long long)st[i]);
+    return SAGE_OK;
+}
+
+sage_status_t check_dev(const void *p, const char *name, size_t align = 16) {
+    if (!p) return fail(SAGE_ERR_INVALID_ARG, "%s is null", name);
+    if (reinterpret_cast<uintptr_t>(p) % align)
+        return fail(SAGE_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+    return SAGE_OK;
+}
+
+Src src(const void *p, const int64_t *st) { return Src{static_cast<const uint16_t *>(p), st[0], st[1], st[2]}; }
+Dst dst(void *p, const int64_t *st) { return Dst{static_cast<uint16_t *>(p), st[0], st[1], st[2]}; }
+
+// Scratch obtained for one call: the caller's buffer or a stream-ordered allocation.
+struct Scratch {
+    void *ptr = nullptr;
+    bool owned = false;
+    cudaStream_t st = nullptr;
+    ~Scratch() {
+        if (owned && ptr) cudaFreeAsync(ptr, st);
+    }
+};
+
+sage_status_t get_scratch(Scratch &s, void *ws, size_t ws_bytes, size_t need, cudaStream_t st) {
+    s.st = st;
+    if (ws) {
+        if (ws_bytes < need)
+            return fail(SAGE_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu required", ws_bytes, need);
+        if (reinterpret_cast<uintptr_t>(ws) % 256) return fail(SAGE_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+        s.ptr = ws;
+        return SAGE_OK;
+    }
+    cudaError_t e = cudaMallocAsync(&s.ptr, need, st);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaMallocAsync(workspace)");
+    s.owned = true;
+    return SAGE_OK;
+}
+
+}  // namespace
+
+size_t stats_ws_bytes(const Shape &s) {
+    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d * sizeof(float);
+    const size_t per = (size_t)s.BH() * s.d * sizeof(float);
+    return 2 * up(part) + 2 * up(per);
+}
+
+StatsWs carve_stats_ws(void *base, const Shape &s) {
+    char *p = static_cast<char *>(base);
+    const size_t part = up((size_t)s.BH() * s.n_chunks() * s.d * sizeof(float));
+    const size_t per = up((size_t)s.BH() * s.d * sizeof(float));
+    StatsWs w;
+    w.ksum_part = reinterpret_cast<float *>(p);
+    w.vmax_part = reinterpret_cast<float *>(p + part);
+    w.k_mean = reinterpret_cast<float *>(p + 2 * part);
+    w.v_inv = reinterpret_cast<float *>(p + 2 * part + per);
+    return w;
+}
+
+size_t codes_bytes(const Shape &s) {
+    const size_t codes = up((size_t)s.BH() * s.n_pad() * s.d);
+    return 3 * codes + up((size_t)s.BH() * s.n_qblocks() * 4) + up((size_t)s.BH() * s.n_kblocks() * 4) +
+           up((size_t)s.BH() * s.d * 4);
+}
+
+Codes carve_codes(void *base, const Shape &s) {
+    char *p = static_cast<char *>(base);
+    const size_t codes = up((size_t)s.BH() * s.n_pad() * s.d);
+    Codes c;
+    c.q_i8 = reinterpret_cast<int8_t *>(p);
+    c.k_i8 = reinterpret_cast<int8_t *>(p + codes);
+    c.v_t8 = reinterpret_cast<uint8_t *>(p + 2 * codes);
+    p += 3 * codes;
+    c.q_scale = reinterpret_cast<float *>(p);
+    p += up((size_t)s.BH() * s.n_qblocks() * 4);
+    c.k_scale = reinterpret_cast<float *>(p);
+    p += up((size_t)s.BH() * s.n_kblocks() * 4);
+    c.v_scale = reinterpret_cast<float *>(p);
+    return c;
+}
+
+}  // namespace sage
+
+using namespace sage;
+
+extern "C" {
+
+const char *sage_status_string(sage_status_t status) {
+    switch (status) {
+        case SAGE_OK: return "SAGE_OK";
+        case SAGE_ERR_INVALID_ARG: return "SAGE_ERR_INVALID_ARG";
+        case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
+        case SAGE_ERR_WORKSPACE: return "SAGE_ERR_WORKSPACE";
+        case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
+        case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+    }
+    return "SAGE_ERR_UNKNOWN";
+}
+
+const char *sage_last_error_message(void) { return g_last_error.c_str(); }
+
+sage_status_t sage_check(sage_stream_t stream) {
+    unsigned v = 0;
+    cudaError_t e = read_and_clear_device_error(&v, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "sage_check");
+    if (v & kErrTimeoutBit) return fail(SAGE_ERR_TIMEOUT, "a kernel gave up on a bounded wait (error word 0x%x)", v);
+    return SAGE_OK;
+}
+
+size_t sage_quant_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    return stats_ws_bytes(Shape{B, H, N, d});
+}
+
+size_t sage_attn_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    const Shape s{B, H, N, d};
+    return up(codes_bytes(s)) + stats_ws_bytes(s);
+}
+
+sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4], const void *k_bf16,
+                            const int64_t k_stride[4], int B, int H, int N, int d, int8_t *q_i8, float *q_scale,
+                            int8_t *k_i8, float *k_scale, float *k_mean, void *workspace, size_t workspace_bytes,
+                            sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_view(q_bf16, q_stride, "q")) ||
+        (r = check_view(k_bf16, k_stride, "k")) || (r = check_dev(q_i8, "q_i8", 16)) ||
+        (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(q_scale, "q_scale", 4)) ||
+        (r = check_dev(k_scale, "k_scale", 4)))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    if ((r = get_scratch(scr, workspace, workspace_bytes, stats_ws_bytes(s), st))) return r;
+    const StatsWs ws = carve_stats_ws(scr.ptr, s);
+    const Src qs = src(q_bf16, q_stride), ks = src(k_bf16, k_stride);
+    Codes c{};
+    c.q_i8 = q_i8;
+    c.q_scale = q_scale;
+    c.k_i8 = k_i8;
+    c.k_scale = k_scale;
+    cudaError_t e = launch_stats(s, &ks, nullptr, ws, k_mean, nullptr, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, &qs, &ks, nullptr, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    return SAGE_OK;
+}
+
+sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B, int H, int N, int d, uint8_t *v_t8,
+                           float *v_scale, void *workspace, size_t workspace_bytes, sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_view(v_bf16, v_stride, "v")) ||
+        (r = check_dev(v_t8, "v_t8", 16)) || (r = check_dev(v_scale, "v_scale", 4)))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    if ((r = get_scratch(scr, workspace, workspace_bytes, stats_ws_bytes(s), st))) return r;
+    const StatsWs ws = carve_stats_ws(scr.ptr, s);
+    const Src vs = src(v_bf16, v_stride);
+    Codes c{};
+    c.v_t8 = v_t8;
+    c.v_scale = v_scale;
+    cudaError_t e = launch_stats(s, nullptr, &vs, ws, nullptr, v_scale, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, nullptr, nullptr, &vs, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    return SAGE_OK;
+}
+
+static sage_status_t check_scale(float sm_scale) {
+    if (!std::isfinite(sm_scale) || !(sm_scale > 0.f))
+        return fail(SAGE_ERR_INVALID_ARG, "sm_scale=%g must be finite and > 0", (double)sm_scale);
+    return SAGE_OK;
+}
+
+sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8, const float *k_scale,
+                                  const uint8_t *v_t8, const float *v_scale, void *out, const int64_t o_stride[4],
+                                  int B, int H, int N, int d, float sm_scale, sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_dev(q_i8, "q_i8", 16)) ||
+        (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(v_t8, "v_t8", 16)) ||
+        (r = check_dev(q_scale, "q_scale", 4)) || (r = check_dev(k_scale, "k_scale", 4)) ||
+        (r = check_dev(v_scale, "v_scale", 4)) || (r = check_view(out, o_stride, "out")))
+        return r;
+    const Shape s{B, H, N, d};
+    Codes c;
+    c.q_i8 = const_cast<int8_t *>(q_i8);
+    c.q_scale = const_cast<float *>(q_scale);
+    c.k_i8 = const_cast<int8_t *>(k_i8);
+    c.k_scale = const_cast<float *>(k_scale);
+    c.v_t8 = const_cast<uint8_t *>(v_t8);
+    c.v_scale = const_cast<float *>(v_scale);
+    cudaError_t e = launch_attention(s, c, dst(out, o_stride), sm_scale, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+    return SAGE_OK;
+}
+
+sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
+                            const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4], int B,
+                            int H, int N, int d, float sm_scale, void *workspace, size_t workspace_bytes,
+                            sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
+        (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
+        (r = check_view(out, o_stride, "out")))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    const size_t cb = up(codes_bytes(s));
+    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + stats_ws_bytes(s), st))) return r;
+    const Codes c = carve_codes(scr.ptr, s);
+    const StatsWs ws = carve_stats_ws(static_cast<char *>(scr.ptr) + cb, s);
+    const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
+    cudaError_t e = launch_stats(s, &ks, &vs, ws, nullptr, c.v_scale, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, &qs, &ks, &vs, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if ((e = launch_attention(s, c, dst(out, o_stride), sm_scale, st)) != cudaSuccess)
+        return cuda_fail(e, "attention kernel");
+    return SAGE_OK;
+}
+
+sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4], const void *k,
+                                      const int64_t k_stride[4], const void *v, const int64_t v_stride[4], void *out,
+                                      const int64_t o_stride[4], int B, int H, int N, int d, float sm_scale,
+                                      sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
+        (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
+        (r = check_view(out, o_stride, "out")))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaError_t e = launch_dense_ref(s, src(q, q_stride), src(k, k_stride), src(v, v_stride), dst(out, o_stride),
+                                     sm_scale, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dense reference kernel");
+    return SAGE_OK;
+}
+
+sage_status_t sage_debug_qk_tile(const int8_t *q_i8, const int8_t *k_i8, int B, int H, int N, int d, int b, int h,
+                                 int q_tile, int kv_tile, int32_t *s_out, sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_dev(q_i8, "q_i8", 16)) || (r = check_dev(k_i8, "k_i8", 16)) ||
+        (r = check_dev(s_out, "s_out", 16)))
+        return r;
+    const Shape s{B, H, N, d};
+    if (b < 0 || b >= B || h < 0 || h >= H || q_tile < 0 || q_tile >= s.n_qblocks() || kv_tile < 0 ||
+        kv_tile >= s.n_qblocks())
+        return fail(SAGE_ERR_INVALID_ARG, "tile (b=%d h=%d q_tile=%d kv_tile=%d) outside the tensor", b, h, q_tile,
+                    kv_tile);
+    cudaError_t e = launch_debug_qk_tile(s, q_i8, k_i8, b * H + h, q_tile, kv_tile, s_out,
+                                         reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "debug S tile");
+    return SAGE_OK;
+}
+
+}  // extern "C"

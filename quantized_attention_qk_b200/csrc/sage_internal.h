@@ -1,0 +1,75 @@
+// sage_internal.h -- host-side plumbing shared by the library's translation
+// units (not installed; the public interface is include/sage.h).
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace sage {
+
+constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
+constexpr int kKBlock = 64;        // K tokens per quantization block
+constexpr int kKvTile = 128;       // keys per attention KV tile (two K blocks)
+constexpr int kStatsChunk = 512;   // tokens per CTA of the statistics pass
+constexpr unsigned kErrTimeoutBit = 1u;  // device error word: a bounded wait gave up
+
+// A bf16 [B,H,N,d] tensor given by base pointer and element strides (c stride 1).
+struct Src {
+    const uint16_t *p;
+    int64_t sb, sh, sn;
+};
+struct Dst {
+    uint16_t *p;
+    int64_t sb, sh, sn;
+};
+
+struct Shape {
+    int B, H, N, d;
+    int BH() const { return B * H; }
+    int n_pad() const { return ((N + kQBlock - 1) / kQBlock) * kQBlock; }
+    int n_qblocks() const { return n_pad() / kQBlock; }
+    int n_kblocks() const { return n_pad() / kKBlock; }
+    int n_chunks() const { return (N + kStatsChunk - 1) / kStatsChunk; }
+};
+
+// Scratch of the quantize pass: per-chunk partials and the finished statistics.
+struct StatsWs {
+    float *ksum_part;  // [BH][chunks][d]
+    float *vmax_part;  // [BH][chunks][d]
+    float *k_mean;     // [BH][d]
+    float *v_inv;      // [BH][d]  448 / amax (0 for an all-zero channel)
+};
+
+// Codes and scales consumed by the attention kernel.
+struct Codes {
+    int8_t *q_i8;      // [BH][N_pad][d]
+    float *q_scale;    // [BH][N_pad/128]
+    int8_t *k_i8;      // [BH][N_pad][d]
+    float *k_scale;    // [BH][N_pad/64]
+    uint8_t *v_t8;     // [BH][d][N_pad]  e4m3 bits
+    float *v_scale;    // [BH][d]
+};
+
+size_t stats_ws_bytes(const Shape &s);
+StatsWs carve_stats_ws(void *base, const Shape &s);
+size_t codes_bytes(const Shape &s);
+Codes carve_codes(void *base, const Shape &s);
+
+// Quantize pass launchers (sage_quant.cu).  `user_k_mean` may be null.
+cudaError_t launch_stats(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, float *user_k_mean,
+                         float *v_scale, cudaStream_t st);
+cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
+                         const Codes &c, cudaStream_t st);
+
+// Attention launchers (sage_attn.cu).
+cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);
+cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,
+                                 int kv_tile, int32_t *s_out, cudaStream_t st);
+cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st);
+
+// Dense fp32 reference (sage_dense_ref.cu).
+cudaError_t launch_dense_ref(const Shape &s, const Src &q, const Src &k, const Src &v, const Dst &out,
+                             float sm_scale, cudaStream_t st);
+
+}  // namespace sage

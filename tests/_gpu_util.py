@@ -1,0 +1,63 @@
+"""Helpers for the GPU parity tests: run the oracle on chosen heads/rows of the
+same seeded inputs and compare element by element."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+
+# Tolerances of the quantized path against the quant-emulation oracle
+# (relative L2 over the compared elements, and max absolute difference).
+REL_L2_TOL = 2e-3
+MAX_ABS_TOL = 1e-2
+
+
+def bf16_to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def sample_rows(N: int, n: int, seed: int) -> np.ndarray:
+    """First, last, the ragged tail tile and random rows (sorted, unique)."""
+    rng = np.random.default_rng(seed)
+    tail0 = (N - 1) // 128 * 128
+    fixed = [0, 1, 127, 128, N - 1, tail0, min(N - 1, tail0 + 1), N // 2]
+    rnd = rng.choice(N, size=min(N, n), replace=False)
+    rows = np.unique(np.clip(np.array(fixed + list(rnd)), 0, N - 1))
+    return rows.astype(np.int32)
+
+
+def oracle_quant_rows(q, k, v, sm_scale, heads, rows):
+    """Oracle quant-emulation outputs for the listed (b,h) heads and rows.
+    q,k,v are CPU bf16 [B,H,N,d].  Returns dict (b,h) -> (f64 [R,d], bf16-as-f64 [R,d])."""
+    res = {}
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        f64, bits = oracle.attn_quant(q[sl], k[sl], v[sl], sm_scale, rows=rows)
+        res[(b, h)] = (f64[0, 0], oracle.bf16_bits_to_f64(bits[0, 0]))
+    return res
+
+
+def oracle_exact_rows(q, k, v, sm_scale, heads, rows):
+    res = {}
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        res[(b, h)] = oracle.attn_exact(q[sl], k[sl], v[sl], sm_scale, rows=rows)[0, 0]
+    return res
+
+
+def compare(got: np.ndarray, want: np.ndarray):
+    """(relative L2, max abs) of got vs want."""
+    diff = got - want
+    rel = float(np.linalg.norm(diff) / max(np.linalg.norm(want), 1e-30))
+    mx = float(np.max(np.abs(diff))) if diff.size else 0.0
+    return rel, mx
+
+
+def gather(out_gpu: torch.Tensor, heads, rows):
+    o = out_gpu.detach().float().cpu()
+    return {(b, h): o[b, h, rows].numpy().astype(np.float64) for (b, h) in heads}
+
+
+def stack(d: dict, heads):
+    return np.stack([d[x] for x in heads])

@@ -1,0 +1,86 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function include/sage.h declares, sizes its scratch as documented, and
+rejects bad arguments before touching a device (only validation paths run)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_attention_qk_b200 as sage
+from quantized_attention_qk_b200 import build as sage_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    sage_build.build()
+    return sage.lib()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "sage.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(sage_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("sage_quant_qk", "sage_attn_fwd", "sage_attn_dense_ref_gpu", "sage_debug_qk_tile",
+                     "sage_attn_workspace_bytes", "sage_status_string", "sage_last_error_message"):
+        assert required in names
+
+
+def test_library_exports_every_declared_function(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in sage.SAGE_STATUS.items():
+        assert L.sage_status_string(code).decode() == name
+
+
+def test_workspace_sizes(L):
+    # codes: 3 * BH * N_pad * d bytes plus scales and statistics
+    for (B, H, N, d) in [(1, 2, 256, 64), (1, 24, 4608, 128), (1, 40, 34020, 128)]:
+        npd = -(-N // 128) * 128
+        ws = sage.sage_attn_workspace_bytes(B, H, N, d)
+        assert ws >= 3 * B * H * npd * d
+        assert ws <= 3 * B * H * npd * d + 64 * 1024 * 1024
+        assert sage.sage_quant_workspace_bytes(B, H, N, d) > 0
+    assert sage.sage_attn_workspace_bytes(1, 1, 128, 96) == 0
+    assert sage.sage_attn_workspace_bytes(1, 1, 0, 64) == 0
+
+
+def _call_fwd(L, q=16 * 4096, strides=(8 * 4096, 4096 * 8, 8 * 8, 1), B=1, H=1, N=128, d=64, scale=0.125):
+    st = (ctypes.c_int64 * 4)(*strides)
+    p = ctypes.c_void_p(q)
+    return L.sage_attn_fwd(p, st, p, st, p, st, p, st, B, H, N, d, ctypes.c_float(scale), None, 0, None)
+
+
+def test_validation_rejects_before_launch(L):
+    # every case below fails in argument checking, before any CUDA call
+    assert _call_fwd(L, d=96) == 2                       # unsupported head dim
+    assert b"d=96" in L.sage_last_error_message()
+    assert _call_fwd(L, N=0) == 1
+    assert _call_fwd(L, q=0) == 1                          # null pointer
+    assert _call_fwd(L, q=16 * 4096 + 2) == 1              # not 16-byte aligned
+    assert _call_fwd(L, strides=(8 * 4096, 4096 * 8, 8 * 8, 2)) == 1   # channel stride != 1
+    assert _call_fwd(L, strides=(8 * 4096, 4096 * 8, 65, 1)) == 1      # row stride not a multiple of 8
+    assert _call_fwd(L, scale=float("nan")) == 1
+    assert _call_fwd(L, scale=0.0) == 1
+    assert _call_fwd(L, scale=-1.0) == 1
+
+
+def test_debug_tile_rejects_out_of_range(L):
+    p = ctypes.c_void_p(16 * 4096)
+    assert L.sage_debug_qk_tile(p, p, 1, 1, 200, 64, 0, 0, 2, 0, p, None) == 1   # q_tile 2 of 2 tiles
+    assert L.sage_debug_qk_tile(p, p, 1, 1, 200, 64, 1, 0, 0, 0, p, None) == 1   # b out of range
+
+
+def test_binding_raises_without_fallback(L):
+    with pytest.raises(sage.SageError) as e:
+        sage._raise(2)
+    assert e.value.status == 2

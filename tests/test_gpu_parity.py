@@ -1,0 +1,265 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded inputs.
+
+  * quantize pass: Q codes/scales and V codes/scales bit-exact; K mean within
+    fp32 summation error; K codes equal except +-1 flips at near ties that the
+    fp32-vs-fp64 smoothing mean can move.
+  * S = Q K^T tiles from the tcgen05 INT8 path: bit-exact against the integer
+    products of the GPU's own codes (closed form).
+  * attention output against the quant-emulation oracle: relative L2 <= 2e-3
+    and max |diff| <= 1e-2 (tolerances of the scheme's specification).
+  * attention output against exact fp64 attention: within the scheme's own
+    error (the oracle's quant-vs-exact gap) plus a small margin.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_qk_b200 as sage
+from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv, tiny_custom
+from tests import _gpu_util as U
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from quantized_attention_qk_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _inputs(w):
+    q, k, v, _ = make_qkv(w)                  # CPU copies for the oracle
+    qd, kd, vd, bufs = make_qkv(w, device=DEV)
+    return (q, k, v), (qd, kd, vd), bufs
+
+
+def _check_attn(w, heads=None, nrows=None, seed=0):
+    (q, k, v), (qd, kd, vd), _ = _inputs(w)
+    heads = heads or [(b, h) for b in range(w.B) for h in range(w.H)]
+    rows = np.arange(w.N, dtype=np.int32) if nrows is None else U.sample_rows(w.N, nrows, seed)
+    out = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    got = U.stack(U.gather(out, heads, rows), heads)
+    ref = U.oracle_quant_rows(q, k, v, w.sm_scale, heads, rows)
+    want_bf16 = np.stack([ref[x][1] for x in heads])
+    rel, mx = U.compare(got, want_bf16)
+    assert np.isfinite(got).all()
+    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL, (w.name, rel, mx)
+    return got, (q, k, v), heads, rows
+
+
+# --------------------------------------------------------------------------- quantize pass
+
+@pytest.mark.parametrize("name", ["tiny", "flux"])
+def test_quant_codes_match_oracle(name):
+    w = WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), _ = _inputs(w)
+    r = sage.sage_quant_qk(qd, kd)
+    v_t8, v_scale = sage.sage_quant_v(vd)
+    torch.cuda.synchronize()
+    N, npd = w.N, sage.n_pad(w.N)
+    heads = [(0, h) for h in range(min(w.H, 3))]
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        o = oracle.quantize(q[sl], k[sl], v[sl])
+        gq = r["q_i8"][b, h].cpu().numpy()
+        np.testing.assert_array_equal(gq[:N], o["q_i8"][0, 0])
+        assert (gq[N:] == 0).all()
+        nqb = -(-N // 128)
+        np.testing.assert_array_equal(r["q_scale"][b, h, :nqb].cpu().numpy(), o["q_scale"][0, 0])
+        np.testing.assert_allclose(r["k_mean"][b, h].cpu().numpy(), o["k_mean"][0, 0], rtol=2e-6, atol=1e-6)
+        nkb = -(-N // 64)
+        np.testing.assert_allclose(r["k_scale"][b, h, :nkb].cpu().numpy(), o["k_scale"][0, 0], rtol=1e-5)
+        gk = r["k_i8"][b, h].cpu().numpy().astype(np.int64)
+        dk = gk[:N] - o["k_i8"][0, 0].astype(np.int64)
+        assert np.abs(dk).max() <= 1 and (dk != 0).mean() < 1e-3, (np.abs(dk).max(), (dk != 0).mean())
+        assert (gk[N:] == 0).all()
+        gv = v_t8[b, h].cpu().numpy()            # [d, N_pad]
+        np.testing.assert_array_equal(gv[:, :N].T, o["v_e4m3"][0, 0])
+        assert (gv[:, N:] == 0).all()
+        np.testing.assert_array_equal(v_scale[b, h].cpu().numpy(), o["v_scale"][0, 0])
+
+
+# --------------------------------------------------------------------------- S tiles
+
+@pytest.mark.parametrize("d,N", [(64, 256), (128, 300), (128, 4608)])
+def test_debug_qk_tile_is_exact_integer_product(d, N):
+    w = tiny_custom(1, 2, N, d, seed=100 + N, bias_sigma=3.0, outlier_frac=0.02)
+    _, (qd, kd, vd), _ = _inputs(w)
+    r = sage.sage_quant_qk(qd, kd)
+    qi = r["q_i8"].cpu().numpy()
+    ki = r["k_i8"].cpu().numpy()
+    nt = sage.n_pad(N) // 128
+    tiles = {(0, 0), (nt - 1, nt - 1), (0, nt - 1), (nt - 1, 0)}
+    for (qt, kt) in sorted(tiles):
+        for h in range(2):
+            s = sage.sage_debug_qk_tile(r["q_i8"], r["k_i8"], N, 0, h, qt, kt).cpu().numpy()
+            want = oracle.int8_gemm_nt(qi[0, h, qt * 128:(qt + 1) * 128], ki[0, h, kt * 128:(kt + 1) * 128])
+            np.testing.assert_array_equal(s, want)
+
+
+# --------------------------------------------------------------------------- attention output
+
+def test_tiny_all_rows():
+    _check_attn(WORKLOADS["tiny"])
+
+
+def test_sdxl_sampled():
+    _check_attn(WORKLOADS["sdxl"], heads=[(0, 0), (3, 9), (2, 4)], nrows=96)
+
+
+def test_flux_full_size_sampled():
+    _check_attn(WORKLOADS["flux"], heads=[(0, 0), (0, 13), (0, 23)], nrows=96)
+
+
+def test_video_full_size_sampled():
+    _check_attn(WORKLOADS["video"], heads=[(0, 0), (0, 39)], nrows=48)
+
+
+@pytest.mark.parametrize("N", [1, 17, 63, 64, 65, 127, 128, 129, 255, 383, 1000])
+@pytest.mark.parametrize("d", [64, 128])
+def test_ragged_and_short_sequences(N, d):
+    _check_attn(tiny_custom(1, 1, N, d, seed=7 * N + d, bias_sigma=2.0))
+
+
+def test_batched_heads_d64():
+    _check_attn(tiny_custom(3, 2, 200, 64, seed=77, bias_sigma=1.0), nrows=None)
+
+
+def test_growing_scores_exercise_the_rescale():
+    """Keys whose scores grow along the sequence: the running max moves at
+    almost every step, so O and l are rescaled many times."""
+    N, d = 1024, 128
+    g = torch.Generator().manual_seed(9)
+    q = torch.randn(1, 1, N, d, generator=g)
+    k = torch.randn(1, 1, N, d, generator=g) * torch.linspace(0.2, 4.0, N).view(1, 1, N, 1)
+    v = torch.randn(1, 1, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    out = sage.sage_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV))
+    torch.cuda.synchronize()
+    rows = np.arange(N, dtype=np.int32)
+    ref = U.oracle_quant_rows(q, k, v, 1 / math.sqrt(d), [(0, 0)], rows)[(0, 0)][1]
+    rel, mx = U.compare(U.bf16_to_f64(out[0, 0]), ref)
+    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL, (rel, mx)
+
+
+def test_zero_query_gives_mean_of_quantized_v():
+    N, d = 300, 64
+    g = torch.Generator().manual_seed(10)
+    q = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    k = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    out = sage.sage_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV))
+    torch.cuda.synchronize()
+    ref = U.oracle_quant_rows(q, k, v, 0.125, [(0, 0)], np.arange(N, dtype=np.int32))[(0, 0)][1]
+    rel, mx = U.compare(U.bf16_to_f64(out[0, 0]), ref)
+    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL
+    # every row is the same (uniform softmax)
+    assert (out[0, 0] == out[0, 0, :1]).all()
+
+
+def test_attention_kernel_on_oracle_codes():
+    """Feed the oracle's own codes and scales to the attention kernel alone: this
+    isolates the tcgen05 attention from the quantize pass."""
+    w = tiny_custom(1, 2, 700, 128, seed=55, bias_sigma=4.0, outlier_frac=0.02)
+    (q, k, v), _, _ = _inputs(w)
+    o = oracle.quantize(q, k, v)
+    N, npd = w.N, sage.n_pad(w.N)
+
+    def pad_rows(a, n):
+        z = np.zeros(a.shape[:2] + (n,) + a.shape[3:], dtype=a.dtype)
+        z[:, :, :a.shape[2]] = a
+        return z
+
+    q_i8 = torch.from_numpy(pad_rows(o["q_i8"], npd)).to(DEV)
+    k_i8 = torch.from_numpy(pad_rows(o["k_i8"], npd)).to(DEV)
+    v_t8 = torch.from_numpy(np.ascontiguousarray(pad_rows(o["v_e4m3"], npd).transpose(0, 1, 3, 2))).to(DEV)
+    qs = np.zeros((1, 2, npd // 128), np.float32); qs[..., :o["q_scale"].shape[-1]] = o["q_scale"]
+    ks = np.zeros((1, 2, npd // 64), np.float32); ks[..., :o["k_scale"].shape[-1]] = o["k_scale"]
+    out = sage.sage_attn_quantized(q_i8, torch.from_numpy(qs).to(DEV), k_i8, torch.from_numpy(ks).to(DEV),
+                                   v_t8, torch.from_numpy(o["v_scale"]).to(DEV), N, w.sm_scale)
+    torch.cuda.synchronize()
+    rows = np.arange(N, dtype=np.int32)
+    ref = U.oracle_quant_rows(q, k, v, w.sm_scale, [(0, 0), (0, 1)], rows)
+    got = U.stack(U.gather(out, [(0, 0), (0, 1)], rows), [(0, 0), (0, 1)])
+    want = np.stack([ref[(0, 0)][1], ref[(0, 1)][1]])
+    rel, mx = U.compare(got, want)
+    assert rel <= 1e-3 and mx <= U.MAX_ABS_TOL, (rel, mx)
+
+
+def test_fused_and_contiguous_layouts_give_identical_bits():
+    w = tiny_custom(1, 3, 500, 128, seed=31, layout="fused", bias_sigma=4.0, outlier_frac=0.01)
+    _, (qd, kd, vd), _ = _inputs(w)
+    out_f = sage.sage_attn_fwd(qd, kd, vd)
+    out_c = sage.sage_attn_fwd(qd.contiguous(), kd.contiguous(), vd.contiguous())
+    torch.cuda.synchronize()
+    assert torch.equal(out_f.view(torch.int16), out_c.view(torch.int16))
+
+
+def test_strided_output_and_explicit_workspace():
+    w = tiny_custom(2, 2, 333, 64, seed=32, bias_sigma=2.0)
+    _, (qd, kd, vd), _ = _inputs(w)
+    ref = sage.sage_attn_fwd(qd, kd, vd)
+    ws = torch.empty(sage.sage_attn_workspace_bytes(2, 2, 333, 64), dtype=torch.uint8, device=DEV)
+    big = torch.zeros(2, 333, 2, 64, dtype=torch.bfloat16, device=DEV)      # [B,N,H,d] storage
+    out = big.permute(0, 2, 1, 3)
+    sage.sage_attn_fwd(qd, kd, vd, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out.contiguous().view(torch.int16), ref.view(torch.int16))
+    small = torch.empty(100, dtype=torch.uint8, device=DEV)
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_attn_fwd(qd, kd, vd, workspace=small)
+    assert e.value.status == 3
+
+
+def test_repeat_calls_are_deterministic():
+    w = WORKLOADS["tiny"]
+    _, (qd, kd, vd), _ = _inputs(w)
+    a = sage.sage_attn_fwd(qd, kd, vd)
+    b = sage.sage_attn_fwd(qd, kd, vd)
+    torch.cuda.synchronize()
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+# --------------------------------------------------------------------------- dense reference and exact
+
+@pytest.mark.parametrize("name", ["tiny", "sdxl"])
+def test_dense_ref_against_exact(name):
+    w = WORKLOADS[name]
+    (q, k, v), (qd, kd, vd), _ = _inputs(w)
+    out = sage.sage_attn_dense_ref_gpu(qd, kd, vd, sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    rows = U.sample_rows(w.N, 64, 3)
+    ex = U.oracle_exact_rows(q, k, v, w.sm_scale, heads, rows)
+    got = U.stack(U.gather(out, heads, rows), heads)
+    want = U.stack(ex, heads)
+    want_bf16 = oracle.bf16_bits_to_f64(oracle.bf16_rne(want)).reshape(want.shape)
+    # only bf16 rounding separates them: at most one bf16 step apart, rarely even that
+    step = np.abs(want_bf16) * 2.0 ** -7 + 1e-30
+    assert np.all(np.abs(got - want_bf16) <= step * 1.01)
+    assert np.mean(got != want_bf16) < 0.02
+    rel, _ = U.compare(got, want)
+    assert rel < 3e-3
+
+
+def test_quantized_against_exact_is_the_schemes_own_error():
+    w = WORKLOADS["flux"]
+    got, (q, k, v), heads, rows = _check_attn(w, heads=[(0, 5)], nrows=64, seed=4)
+    ex = U.stack(U.oracle_exact_rows(q, k, v, w.sm_scale, heads, rows), heads)
+    emu = np.stack([U.oracle_quant_rows(q, k, v, w.sm_scale, heads, rows)[x][1] for x in heads])
+    gpu_err, _ = U.compare(got, ex)
+    emu_err, _ = U.compare(emu, ex)
+    assert gpu_err <= 1.05 * emu_err + 1e-3, (gpu_err, emu_err)
+
+
+def test_device_error_word_is_clear():
+    sage.sage_check()
