@@ -1,0 +1,325 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized attention forward on B200.
+
+One step = one full forward (statistics + quantize + fused attention) of the
+workload, through the C ABI (sage_attn_fwd).  Metric: TOPS = 4*B*H*N^2*d / t.
+
+  python bench.py [--gpus N --steps K --warmup W] [--workload flux|video|...]
+  python bench.py --impl reference ...   # the CPU oracle, timed on the host
+
+N > 1 GPUs (torchrun): every rank runs its own copy of the workload (the heads
+of independent problems; no data-path collective), so the scaling is weak and
+the value is the sum over ranks of the work divided by the slowest rank's time.
+
+Inputs are seeded synthetic tensors (quantized_attention_qk_b200.inputs).  The
+L2 is flushed (a 256 MB write) before every timed step, outside the events.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "quantized attention TOPS (4·B·H·N²·d/t) and ms/call at N=4608 and N=34020, d=128"
+DTYPE = "i8/e4m3"        # QK^T on int8 codes, PV on e4m3 codes; bf16 in and out
+PRIMARY, SECONDARY = "flux", "video"
+PEAK_NOTE = "measured cuBLAS bf16 burst x 2 (nominal 8-bit/bf16 dense ratio)"
+LAUNCHES_PER_STEP = 4    # stats partial, stats final, quantize, attention
+
+
+def _env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def _workload_desc(w):
+    return f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.layout} qkv"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (200 ms) of one GPU while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = float(parts[1])
+            except ValueError:
+                continue
+            for nm, val in zip(names, parts[4:8]):
+                if val.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle baseline
+def cpu_oracle_sample(w, seconds=12.0, seed=0):
+    """Time the CPU oracle's quant emulation on a bounded sample of the workload:
+    whole-slab quantization of one head plus as many query rows of it as fit in
+    about ``seconds``.  Returns (TOPS-equivalent, rows, elapsed, cores)."""
+    import numpy as np
+    import oracle
+    from quantized_attention_qk_b200.inputs import make_qkv
+
+    oracle.build()
+    one = w.with_(B=1, H=1, name=w.name + "-head0")
+    q, k, v, _ = make_qkv(one)
+    rng = np.random.default_rng(seed)
+    rows_done, t_total, batch = 0, 0.0, 4
+    while t_total < seconds:
+        rows = np.sort(rng.choice(w.N, size=batch, replace=False)).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.attn_quant(q, k, v, w.sm_scale, rows=rows)
+        t_total += time.perf_counter() - t0
+        rows_done += batch
+        batch = min(batch * 2, 64)
+    ops = 4.0 * w.N * w.d * rows_done           # both contractions for the sampled rows
+    return ops / t_total / 1e12, rows_done, t_total, 1
+
+
+# --------------------------------------------------------------------------- GPU arm
+def run_gpu(args):
+    import torch
+    import torch.distributed as dist
+
+    import quantized_attention_qk_b200 as sage
+    from quantized_attention_qk_b200 import build as sage_build
+    from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv
+
+    world = _env_int("WORLD_SIZE", 1)
+    rank = _env_int("RANK", 0)
+    local = _env_int("LOCAL_RANK", 0)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    sage_build.build()
+    sage.lib()
+    peaks, peak_kind = _peaks()
+    peak_8bit = 2.0 * float(peaks["bf16_tflops"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def measure(w, steps, warmup):
+        q, k, v, bufs = make_qkv(w, device=dev)
+        out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(sage.sage_attn_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for e in ev:
+            for x in e:
+                x.record()          # create the underlying events
+        for _ in range(warmup):
+            sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        barrier()
+        torch.cuda.synchronize()
+        clk = ClockSampler(local)
+        clk.start()
+        for i in range(steps):
+            flush.zero_()
+            s0, a0, a1, s1 = ev[i]
+            s0.record()
+            sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws, attn_events=(a0, a1))
+            s1.record()
+        torch.cuda.synchronize()
+        barrier()
+        torch.cuda.synchronize()
+        clocks = clk.stop()
+        sage.sage_check()
+        step_ms = [e[0].elapsed_time(e[3]) for e in ev]
+        attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+        total_ms = max_over_ranks(sum(step_ms))
+        attn_avg = max_over_ranks(sum(attn_ms) / steps)
+        # end to end through host memory: pinned input -> device, forward, result -> pinned host
+        host_in = bufs[0].cpu().pin_memory() if w.layout == "fused" else torch.stack(bufs).cpu().pin_memory()
+        out_host = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, pin_memory=True)
+        e2e_steps = max(2, min(steps, 10))
+        for _ in range(2):
+            sage.sage_attn_fwd_host(host_in, w.B, w.H, w.N, w.d, layout=w.layout, sm_scale=w.sm_scale,
+                                    device=dev, out_host=out_host, workspace=ws)
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(e2e_steps):
+            sage.sage_attn_fwd_host(host_in, w.B, w.H, w.N, w.d, layout=w.layout, sm_scale=w.sm_scale,
+                                    device=dev, out_host=out_host, workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+        sage.sage_check()
+        h2d = host_in.numel() * host_in.element_size()
+        d2h = out_host.numel() * out_host.element_size()
+        del q, k, v, bufs, out, ws, host_in
+        torch.cuda.empty_cache()
+        return dict(total_ms=total_ms, attn_ms=attn_avg, e2e_ms=e2e_ms, clocks=clocks, h2d=h2d, d2h=d2h)
+
+    wp = WORKLOADS[args.workload]
+    r = measure(wp, args.steps, args.warmup)
+    ms = r["total_ms"] / args.steps
+    value = world * wp.ops * args.steps / (r["total_ms"] * 1e-3) / 1e12
+    attn_tops = wp.ops / (r["attn_ms"] * 1e-3) / 1e12
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic (seeded N(0,1) Q/K/V, K bias and outlier channels)",
+        "config": {"workload": _workload_desc(wp), "B": wp.B, "H": wp.H, "N": wp.N, "d": wp.d,
+                   "layout": wp.layout, "sm_scale": wp.sm_scale, "parallelism": f"replicas x{world}",
+                   "l2": "flushed before every timed step (256 MB write, outside the events)"},
+        "roofline": {"bound": "tensor", "kernel": "k_attn (fused attention)", "achieved": round(attn_tops, 2),
+                     "peak": round(peak_8bit, 1), "unit": "TFLOP/s", "frac": round(attn_tops / peak_8bit, 4),
+                     "traffic": None, "peak_source": f"{peak_kind}: {PEAK_NOTE}",
+                     "attn_ms": round(r["attn_ms"], 4)},
+        "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
+                "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
+                "api": "sage_attn_fwd_host (pinned host qkv -> device, sage_attn_fwd, bf16 out -> pinned host)"},
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+        "clocks": r["clocks"],
+    }
+    if args.secondary and args.workload != SECONDARY:
+        ws_ = WORKLOADS[SECONDARY]
+        r2 = measure(ws_, max(3, args.steps // 2), args.warmup)
+        k2 = max(3, args.steps // 2)
+        line["secondary"] = {
+            "workload": _workload_desc(ws_), "value": round(world * ws_.ops * k2 / (r2["total_ms"] * 1e-3) / 1e12, 2),
+            "unit": "TOPS", "ms_per_step": round(r2["total_ms"] / k2, 4), "steps": k2,
+            "attn_tops": round(ws_.ops / (r2["attn_ms"] * 1e-3) / 1e12, 2), "attn_ms": round(r2["attn_ms"], 4),
+            "attn_frac": round(ws_.ops / (r2["attn_ms"] * 1e-3) / 1e12 / peak_8bit, 4),
+            "e2e_tops": round(world * ws_.ops / (r2["e2e_ms"] * 1e-3) / 1e12, 2), "clocks": r2["clocks"]}
+        line["gpu_launches"] += LAUNCHES_PER_STEP * k2
+    if rank == 0 and world == 1 and args.cpu_baseline:
+        tops, rows, secs, cores = cpu_oracle_sample(wp, seconds=args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(tops, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+                                "sample": f"{rows} query rows of head 0 of {wp.name} (full-slab quantization "
+                                          f"included), {secs:.1f} s, quant-emulation mode"}
+    if rank == 0:
+        print(json.dumps(line, ensure_ascii=False), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- reference arm (the CPU oracle)
+def run_reference(args):
+    from quantized_attention_qk_b200.inputs import WORKLOADS
+
+    if _env_int("RANK", 0) != 0:
+        return
+    w = WORKLOADS[args.workload]
+    per_step = max(1.0, args.cpu_seconds / max(1, args.steps))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, seconds=0.5)
+    vals, rows_total, secs_total = [], 0, 0.0
+    for i in range(args.steps):
+        tops, rows, secs, cores = cpu_oracle_sample(w, seconds=per_step, seed=i + 1)
+        vals.append(tops)
+        rows_total += rows
+        secs_total += secs
+    value = 4.0 * w.N * w.d * rows_total / secs_total / 1e12
+    sample = (f"{rows_total} query rows of head 0 of {w.name} over {args.steps} steps "
+              f"(full-slab quantization per call), {secs_total:.1f} s")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs_total / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 quant steps)",
+            "data": "synthetic", "config": {"workload": _workload_desc(w), "B": w.B, "H": w.H, "N": w.N, "d": w.d},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line, ensure_ascii=False), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["sage", "reference"], default="sage")
+    ap.add_argument("--workload", default=PRIMARY)
+    ap.add_argument("--no-secondary", dest="secondary", action="store_false")
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -57,8 +57,9 @@
 extern "C" {
 #endif
 
-/* Same handle type as cudaStream_t (the runtime's opaque stream pointer). */
+/* Same handle types as cudaStream_t / cudaEvent_t (the runtime's opaque pointers). */
 typedef struct CUstream_st *sage_stream_t;
+typedef struct CUevent_st *sage_event_t;
 
 typedef enum {
     SAGE_OK = 0,
@@ -155,6 +156,22 @@ sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4],
                             int B, int H, int N, int d, float sm_scale,
                             void *workspace, size_t workspace_bytes,
                             sage_stream_t stream);
+
+/*
+ * sage_attn_fwd_ev -- sage_attn_fwd that also records `attn_begin` / `attn_end`
+ * (CUDA events created by the caller; either may be NULL) on `stream` right
+ * before and right after the fused attention kernel, so a caller can time that
+ * kernel inside the whole forward.  Same arguments, layouts and errors as
+ * sage_attn_fwd, which is this call with two NULL events.
+ */
+sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4],
+                               const void *k, const int64_t k_stride[4],
+                               const void *v, const int64_t v_stride[4],
+                               void *out, const int64_t o_stride[4],
+                               int B, int H, int N, int d, float sm_scale,
+                               void *workspace, size_t workspace_bytes,
+                               sage_stream_t stream,
+                               sage_event_t attn_begin, sage_event_t attn_end);
 
 /*
  * sage_attn_dense_ref_gpu -- plain dense attention on the CUDA cores in fp32

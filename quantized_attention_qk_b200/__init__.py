@@ -50,6 +50,8 @@ _SIGS = {
     "sage_attn_quantized": ([_P, _P, _P, _P, _P, _P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float, _P], _I32),
     "sage_attn_fwd": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
                        _P, _SZ, _P], _I32),
+    "sage_attn_fwd_ev": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                          _P, _SZ, _P, _P, _P], _I32),
     "sage_attn_dense_ref_gpu": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32,
                                  ctypes.c_float, _P], _I32),
     "sage_debug_qk_tile": ([_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
@@ -160,8 +162,10 @@ def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_t8, v_scale, N: int, sm_
     return out
 
 
-def sage_attn_fwd(q, k, v, sm_scale=None, out=None, workspace=None, stream=None):
-    """Quantized attention forward on device tensors; returns bf16 [B,H,N,d]."""
+def sage_attn_fwd(q, k, v, sm_scale=None, out=None, workspace=None, stream=None, attn_events=None):
+    """Quantized attention forward on device tensors; returns bf16 [B,H,N,d].
+    ``attn_events``: optional pair of recorded-once torch.cuda.Event objects that
+    the library records right before / after the fused attention kernel."""
     _check_qkv(q, k, v)
     B, H, N, d = q.shape
     dev = q.device
@@ -170,9 +174,15 @@ def sage_attn_fwd(q, k, v, sm_scale=None, out=None, workspace=None, stream=None)
     if out is None:
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _raise(lib().sage_attn_fwd(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
-                               _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                               _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    if attn_events is None:
+        _raise(lib().sage_attn_fwd(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                   _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                   _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    else:
+        e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events)
+        _raise(lib().sage_attn_fwd_ev(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                      _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                      _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
     return out
 
 

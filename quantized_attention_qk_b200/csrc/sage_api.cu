@@ -250,10 +250,10 @@ sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale, cons
     return SAGE_OK;
 }
 
-sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
-                            const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4], int B,
-                            int H, int N, int d, float sm_scale, void *workspace, size_t workspace_bytes,
-                            sage_stream_t stream) {
+sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
+                               const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4], int B,
+                               int H, int N, int d, float sm_scale, void *workspace, size_t workspace_bytes,
+                               sage_stream_t stream, sage_event_t attn_begin, sage_event_t attn_end) {
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
@@ -270,9 +270,21 @@ sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4], const void
     cudaError_t e = launch_stats(s, &ks, &vs, ws, nullptr, c.v_scale, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
     if ((e = launch_quant(s, &qs, &ks, &vs, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_attention(s, c, dst(out, o_stride), sm_scale, st)) != cudaSuccess)
         return cuda_fail(e, "attention kernel");
+    if (attn_end && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_end), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
     return SAGE_OK;
+}
+
+sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
+                            const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4], int B,
+                            int H, int N, int d, float sm_scale, void *workspace, size_t workspace_bytes,
+                            sage_stream_t stream) {
+    return sage_attn_fwd_ev(q, q_stride, k, k_stride, v, v_stride, out, o_stride, B, H, N, d, sm_scale, workspace,
+                            workspace_bytes, stream, nullptr, nullptr);
 }
 
 sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4], const void *k,

@@ -66,9 +66,12 @@ struct Ctl {
     float v_scale[D];
 };
 
+// At least 120 KB so that a second CTA never shares the SM: each CTA takes
+// all 512 tensor-memory columns.
 template <int D>
 constexpr int smem_bytes() {
-    return Cfg<D>::TILE_BYTES + static_cast<int>(sizeof(Ctl<D>)) + 1024;
+    constexpr int need = Cfg<D>::TILE_BYTES + static_cast<int>(sizeof(Ctl<D>)) + 1024;
+    return need > 120 * 1024 ? need : 120 * 1024;
 }
 
 struct AttnParams {

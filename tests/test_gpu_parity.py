@@ -50,9 +50,9 @@ def _check_attn(w, heads=None, nrows=None, seed=0):
     got = U.stack(U.gather(out, heads, rows), heads)
     ref = U.oracle_quant_rows(q, k, v, w.sm_scale, heads, rows)
     want_bf16 = np.stack([ref[x][1] for x in heads])
-    rel, mx = U.compare(got, want_bf16)
+    ok, rel, mx = U.within_tol(got, want_bf16)
     assert np.isfinite(got).all()
-    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL, (w.name, rel, mx)
+    assert ok, (w.name, rel, mx)
     return got, (q, k, v), heads, rows
 
 
@@ -147,8 +147,8 @@ def test_growing_scores_exercise_the_rescale():
     torch.cuda.synchronize()
     rows = np.arange(N, dtype=np.int32)
     ref = U.oracle_quant_rows(q, k, v, 1 / math.sqrt(d), [(0, 0)], rows)[(0, 0)][1]
-    rel, mx = U.compare(U.bf16_to_f64(out[0, 0]), ref)
-    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL, (rel, mx)
+    ok, rel, mx = U.within_tol(U.bf16_to_f64(out[0, 0]), ref)
+    assert ok, (rel, mx)
 
 
 def test_zero_query_gives_mean_of_quantized_v():
@@ -160,8 +160,8 @@ def test_zero_query_gives_mean_of_quantized_v():
     out = sage.sage_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV))
     torch.cuda.synchronize()
     ref = U.oracle_quant_rows(q, k, v, 0.125, [(0, 0)], np.arange(N, dtype=np.int32))[(0, 0)][1]
-    rel, mx = U.compare(U.bf16_to_f64(out[0, 0]), ref)
-    assert rel <= U.REL_L2_TOL and mx <= U.MAX_ABS_TOL
+    ok, rel, mx = U.within_tol(U.bf16_to_f64(out[0, 0]), ref)
+    assert ok, (rel, mx)
     # every row is the same (uniform softmax)
     assert (out[0, 0] == out[0, 0, :1]).all()
 
@@ -191,8 +191,8 @@ def test_attention_kernel_on_oracle_codes():
     ref = U.oracle_quant_rows(q, k, v, w.sm_scale, [(0, 0), (0, 1)], rows)
     got = U.stack(U.gather(out, [(0, 0), (0, 1)], rows), [(0, 0), (0, 1)])
     want = np.stack([ref[(0, 0)][1], ref[(0, 1)][1]])
-    rel, mx = U.compare(got, want)
-    assert rel <= 1e-3 and mx <= U.MAX_ABS_TOL, (rel, mx)
+    ok, rel, mx = U.within_tol(got, want, rel_tol=1e-3)
+    assert ok, (rel, mx)
 
 
 def test_fused_and_contiguous_layouts_give_identical_bits():
