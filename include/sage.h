@@ -112,6 +112,34 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4],
                             sage_stream_t stream);
 
 /*
+ * sage_quant_qk_noalloc -- sage_quant_qk for callers that cannot allocate device
+ * memory while they run: an engine or server plugin whose device memory is
+ * budgeted up front and whose execution path forbids cudaMalloc /
+ * cudaMallocAsync, or code whose allocator belongs to a host framework.  The
+ * pages have no counterpart of this entry point; it changes only where the
+ * pass's scratch lives.
+ *   Same arguments, outputs and results as sage_quant_qk, without the
+ *   workspace.  The statistics scratch is a fixed array of
+ *   SAGE_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library's device memory;
+ *   every GPU that loads the library holds it until the process exits.  A shape
+ *   whose scratch (sage_quant_workspace_bytes) exceeds it is rejected with
+ *   SAGE_ERR_WORKSPACE before anything is launched.  The call allocates nothing.
+ *   The first call on each device looks up the array's device address (with
+ *   that device current); make that first call before any stream capture.
+ *   All calls on a device share the array: calls that may overlap on the GPU
+ *   (different streams without ordering) race and must be serialized by the
+ *   caller.  The array keeps the last call's contents; nothing in it needs to
+ *   start at zero.
+ */
+#define SAGE_NOALLOC_SCRATCH_BYTES (4u << 20)
+sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t q_stride[4],
+                                    const void *k_bf16, const int64_t k_stride[4],
+                                    int B, int H, int N, int d,
+                                    int8_t *q_i8, float *q_scale,
+                                    int8_t *k_i8, float *k_scale, float *k_mean,
+                                    sage_stream_t stream);
+
+/*
  * sage_quant_v -- V to FP8 e4m3 with one scale per (b,h,channel) ([H3] "FP8 for
  * PV"; reading C7):  amax_c = max_n |V|;  v_scale = amax_c/448;
  * v_t8[b,h,c,n] = e4m3_rn_satfinite(V * (448/amax_c)).

@@ -19,7 +19,7 @@ import torch
 
 __all__ = [
     "SageError", "lib", "sage_attn_fwd", "sage_attn_quantized", "sage_quant_qk", "sage_quant_v",
-    "sage_attn_dense_ref_gpu", "sage_debug_qk_tile", "sage_attn_workspace_bytes",
+    "sage_attn_dense_ref_gpu", "sage_debug_qk_tile", "sage_quant_qk_noalloc", "sage_attn_workspace_bytes",
     "sage_quant_workspace_bytes", "sage_check", "sage_attn_fwd_host", "n_pad",
 ]
 
@@ -46,6 +46,7 @@ _SIGS = {
     "sage_attn_workspace_bytes": ([_I32] * 4, _SZ),
     "sage_quant_workspace_bytes": ([_I32] * 4, _SZ),
     "sage_quant_qk": ([_P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _SZ, _P], _I32),
+    "sage_quant_qk_noalloc": ([_P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P], _I32),
     "sage_quant_v": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _SZ, _P], _I32),
     "sage_attn_quantized": ([_P, _P, _P, _P, _P, _P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float, _P], _I32),
     "sage_attn_fwd": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
@@ -129,6 +130,28 @@ def sage_quant_qk(q, k, workspace=None, stream=None):
     _raise(lib().sage_quant_qk(_ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
                                _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]), _ptr(r["k_scale"]),
                                _ptr(r["k_mean"]), _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    return r
+
+
+def sage_quant_qk_noalloc(q, k, out=None, stream=None):
+    """sage_quant_qk without a workspace and without any device allocation in
+    the library: its statistics scratch is a fixed 4 MiB array in the library's
+    device memory (shared by all calls on a device; calls that overlap on the
+    GPU race).  ``out`` optionally supplies the output dict (same keys/shapes as
+    sage_quant_qk returns) so that the caller owns every buffer."""
+    _check_qkv(q, k)
+    B, H, N, d = q.shape
+    dev = q.device
+    npd = n_pad(N)
+    r = out if out is not None else dict(
+        q_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
+        q_scale=torch.empty(B, H, npd // Q_BLOCK, dtype=torch.float32, device=dev),
+        k_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
+        k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
+        k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev))
+    _raise(lib().sage_quant_qk_noalloc(_ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
+                                       _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]), _ptr(r["k_scale"]),
+                                       _ptr(r["k_mean"]), _stream(stream, dev)))
     return r
 
 

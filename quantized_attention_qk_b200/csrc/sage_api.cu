@@ -95,6 +95,15 @@ sage_status_t get_scratch(Scratch &s, void *ws, size_t ws_bytes, size_t need, cu
 
 }  // namespace
 
+void set_last_error(const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+}
+
 size_t stats_ws_bytes(const Shape &s) {
     const size_t part = (size_t)s.BH() * s.n_chunks() * s.d * sizeof(float);
     const size_t per = (size_t)s.BH() * s.d * sizeof(float);

@@ -51,6 +51,9 @@ struct Codes {
     float *v_scale;    // [BH][d]
 };
 
+// Record the calling thread's error message (what sage_last_error_message returns).
+void set_last_error(const char *fmt, ...);
+
 size_t stats_ws_bytes(const Shape &s);
 StatsWs carve_stats_ws(void *base, const Shape &s);
 size_t codes_bytes(const Shape &s);

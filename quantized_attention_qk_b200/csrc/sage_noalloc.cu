@@ -1,0 +1,78 @@
+// sage_noalloc.cu -- sage_quant_qk_noalloc: the smoothing + Q/K quantization
+// pass for callers that may not allocate device memory while they run (an
+// engine or server plugin whose device memory is budgeted up front and whose
+// execution path forbids cudaMalloc / cudaMallocAsync, or code whose allocator
+// belongs to a host framework).  The pass needs scratch for its per-chunk
+// statistics; here that scratch is a fixed array in the library's own device
+// memory instead of a caller buffer or a stream-ordered allocation.
+//
+// The array is loaded with the module, so every GPU that loads the library
+// holds it (kNoAllocScratchBytes) until the process exits.  All calls on one
+// device share it: calls that overlap on the GPU (e.g. on two streams without
+// ordering between them) race on it and must be serialized by the caller.
+// It keeps the last call's contents; every entry a call reads is written
+// earlier in the same call, so nothing has to start at zero.
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "sage.h"
+#include "sage_internal.h"
+
+namespace sage {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = SAGE_NOALLOC_SCRATCH_BYTES;
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (with that device current).  Host code cannot use the symbol
+// itself: on the host it only names a stand-in, not device memory.
+cudaError_t scratch_for_current_device(void **out) {
+    static std::mutex mu;
+    static void *ptrs[kMaxDevices] = {nullptr};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        ptrs[dev] = p;
+    }
+    *out = ptrs[dev];
+    return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace sage
+
+extern "C" sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t q_stride[4], const void *k_bf16,
+                                               const int64_t k_stride[4], int B, int H, int N, int d, int8_t *q_i8,
+                                               float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
+                                               sage_stream_t stream) {
+    using namespace sage;
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128))  // reported by the shape check, before any allocation
+        return sage_quant_qk(q_bf16, q_stride, k_bf16, k_stride, B, H, N, d, q_i8, q_scale, k_i8, k_scale,
+                             k_mean, nullptr, 0, stream);
+    const Shape s{B, H, N, d};
+    const size_t need = stats_ws_bytes(s);
+    if (need > kNoAllocScratchBytes) {
+        set_last_error("sage_quant_qk_noalloc: this shape needs %zu bytes of scratch; the built-in scratch "
+                       "holds %zu (B*H*ceil(N/512)*d is too large)",
+                       need, kNoAllocScratchBytes);
+        return SAGE_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    cudaError_t e = scratch_for_current_device(&scratch);
+    if (e != cudaSuccess) {
+        set_last_error("sage_quant_qk_noalloc: cudaGetSymbolAddress failed: %s", cudaGetErrorString(e));
+        return SAGE_ERR_CUDA;
+    }
+    return sage_quant_qk(q_bf16, q_stride, k_bf16, k_stride, B, H, N, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+                         scratch, kNoAllocScratchBytes, stream);
+}
