@@ -168,7 +168,9 @@ sage_status_t sage_check(sage_stream_t stream) {
     unsigned v = 0;
     cudaError_t e = read_and_clear_device_error(&v, stream);
     if (e != cudaSuccess) return cuda_fail(e, "sage_check");
-    if (v & kErrTimeoutBit) return fail(SAGE_ERR_TIMEOUT, "a kernel gave up on a bounded wait (error word 0x%x)", v);
+    if (v & kErrTimeoutBit)
+        return fail(SAGE_ERR_TIMEOUT, "a kernel gave up on a bounded wait (error word 0x%x: bit 8+k marks wait site k)",
+                    v);
     return SAGE_OK;
 }
 

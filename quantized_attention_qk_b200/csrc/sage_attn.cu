@@ -1,21 +1,30 @@
 // sage_attn.cu -- fused quantized attention kernel for sm_100a.
 //
-// One CTA computes two 128-query tiles (Q0, Q1) of one (batch, head) against
-// all keys, 128 keys per step, never writing the score matrix out
+// One CTA computes two 128-query tiles of one (batch, head) against all keys,
+// 128 keys per step, never writing the score matrix out
 // ("GitHub榜单静默期：Attention优化从架构转向推理加速", section 2.2).  Scores come
 // from INT8 tensor-core products and P.V from FP8 (e4m3) products
 // ("MiniMax H3 接入 SageAttention 实测加速", section 一).
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax warpgroup of Q tile 0 (one query row per thread)
-//   warps 4-7  softmax warpgroup of Q tile 1
-//   warp  8    TMA producer: Q tiles once, then a ring of (K tile, V^T tile) stages
-//   warp  9    tensor-memory allocator and single-thread tcgen05.mma issuer
-// Tensor memory (512 columns x 128 lanes):
-//   [0,128) S0 int32, [128,256) S1 int32, [256,256+d) O0 fp32, [256+d,256+2d) O1 fp32.
-//   P_t (e4m3, 4 per column) overwrites columns [0,32) of S_t after softmax.
-// Per KV step j the issue order is  PV0(j), S0(j+1), PV1(j), S1(j+1): while one
-// warpgroup runs its softmax the tensor core works on the other tile.
+// Warp roles (384 threads, three warpgroups):
+//   warpgroup t (warps 4t..4t+3), t = 0, 1: softmax of Q tile t, one query row
+//              per thread; the two warpgroups run independently of each other
+//   warp 8     TMA producer: both Q tiles once, then a ring of (K, V^T) stages
+//   warp 9     tensor-memory allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle
+// After set-up the softmax warpgroups raise their register limit to 224 and
+// warpgroup 2 lowers its own to 48 (setmaxnreg).
+// Tensor memory (512 columns x 128 lanes): S0, S1 (int32, 128 columns each) at
+// [0,256), O0, O1 (fp32, d columns each) from 256.
+// P (e4m3) goes to shared memory, two buffers per tile, in the 128-byte-swizzled
+// K-major layout the P.V MMA reads.  A warpgroup releases S(j) as soon as it
+// holds it in registers, so the tensor core computes S(j+1) while the softmax
+// of step j runs.  MMA order per step j:
+//   S0(j+1), S1(j+1)   (each once its tile released S(j) and K(j+1) is loaded)
+//   PV0(j), PV1(j)     (each once its tile posted P(j) and rescaled O)
+// Barriers a waiter tracks by phase parity never get two phases ahead of it:
+// "P ready" has one barrier per P buffer, and the epilogue waits on a barrier
+// committed once after the tile's last PV.
 // Numerics (readings C4-C8): x = S*(sq*sm_scale*log2e*sk) with one sk per
 // 64-key block; running max m' = max(m, ceil(rowmax x)) so that the O / l
 // rescale 2^(m-m') is an exact power of two; P = e4m3(2^(x-m') * 448) computed as
@@ -42,14 +51,20 @@ template <int D>
 struct Cfg {
     static constexpr int BM = 128;                 // queries per tile
     static constexpr int BN = kKvTile;             // keys per step
-    static constexpr int STAGES = D == 128 ? 3 : 4;
+    static constexpr int STAGES = 3;
     static constexpr int Q_BYTES = BM * D;
     static constexpr int K_BYTES = BN * D;
     static constexpr int V_BYTES = D * BN;
-    static constexpr int TILE_BYTES = 2 * Q_BYTES + STAGES * (K_BYTES + V_BYTES);
-    static constexpr uint32_t T_S0 = 0, T_S1 = 128, T_O0 = 256, T_O1 = 256 + D;
+    static constexpr int P_BYTES = BM * BN;        // one P buffer (e4m3)
+    static constexpr int TILE_BYTES = 2 * Q_BYTES + STAGES * (K_BYTES + V_BYTES) + 4 * P_BYTES;
+    static constexpr uint32_t T_O = 256;           // O of tile t at 256 + d t
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;            // three warpgroups
+    static constexpr int LAUNCH_REGS = 168;        // per thread, what 384 threads x 1 block allow
+    static constexpr uint32_t SOFTMAX_REGS = 224;  // warpgroups 0 and 1 after setmaxnreg
+    static constexpr uint32_t OTHER_REGS = 48;     // warpgroup 2 (TMA, MMA, two idle warps)
+    static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= LAUNCH_REGS * THREADS,
+                  "register split exceeds the registers the block is launched with");
 };
 
 template <int D>
@@ -57,9 +72,11 @@ struct Ctl {
     uint64_t q_full;
     uint64_t kv_full[Cfg<D>::STAGES];
     uint64_t kv_empty[Cfg<D>::STAGES];
-    uint64_t s_full[2];
-    uint64_t p_ready[2];
-    uint64_t o_done[2];
+    uint64_t s_full[2];     // per tile: S(j) computed
+    uint64_t s_free[2];     // per tile: the softmax holds S(j) in registers
+    uint64_t p_ready[2][2]; // [tile][P buffer]: P(j) in shared memory and O rescaled
+    uint64_t o_done[2];     // per tile: PV of a step completed
+    uint64_t o_final[2];    // per tile: every PV of the tile completed (committed once)
     uint64_t drain;
     uint32_t tmem_base;
     AbortState abort;
@@ -67,7 +84,7 @@ struct Ctl {
 };
 
 // At least 120 KB so that a second CTA never shares the SM: each CTA takes
-// all 512 tensor-memory columns.
+// all 512 tensor-memory columns.  (The tiles need more than that anyway.)
 template <int D>
 constexpr int smem_bytes() {
     constexpr int need = Cfg<D>::TILE_BYTES + static_cast<int>(sizeof(Ctl<D>)) + 1024;
@@ -94,6 +111,61 @@ __device__ __forceinline__ float exp2_int(float k) {
     return e > 0 ? __int_as_float(e << 23) : 0.f;
 }
 
+// Largest of the 64 scores in a/b (columns col0.. of the step; with MASK,
+// columns at or past n_valid are left out; INT_MIN if none is valid).
+template <bool MASK>
+__device__ __forceinline__ int row_max64(const uint32_t (&a)[32], const uint32_t (&b)[32], int col0, int n_valid) {
+    int m0 = INT_MIN, m1 = INT_MIN;  // two independent chains
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        int a0 = static_cast<int>(a[i]), a1 = static_cast<int>(a[i + 1]);
+        int b0 = static_cast<int>(b[i]), b1 = static_cast<int>(b[i + 1]);
+        if (MASK) {
+            if (col0 + i >= n_valid) a0 = INT_MIN;
+            if (col0 + i + 1 >= n_valid) a1 = INT_MIN;
+            if (col0 + 32 + i >= n_valid) b0 = INT_MIN;
+            if (col0 + 32 + i + 1 >= n_valid) b1 = INT_MIN;
+        }
+        m0 = __vimax3_s32(m0, a0, a1);
+        m1 = __vimax3_s32(m1, b0, b1);
+    }
+    return max(m0, m1);
+}
+
+// 448 * 2^(x - m) for 32 scores, x = S * c: y = float(S) * c + (log2 448 - m)
+// (one FMA per pair), p = 2^y on the MUFU unit.  Accumulates the unrounded p
+// into acc and packs the e4m3 codes four per word into w[0..7] (word j holds
+// keys 4j..4j+3, lowest key in the lowest byte).
+template <bool MASK>
+__device__ __forceinline__ void p_pack32(const uint32_t (&r)[32], float c, float nb, int col0, int n_valid,
+                                         float (&acc)[4], uint32_t *w) {
+#pragma unroll
+    for (int i = 0; i < 32; i += 4) {
+        float y[4], pv[4];
+        ffma2(y[0], y[1], static_cast<float>(static_cast<int>(r[i])), static_cast<float>(static_cast<int>(r[i + 1])),
+              c, c, nb, nb);
+        ffma2(y[2], y[3], static_cast<float>(static_cast<int>(r[i + 2])),
+              static_cast<float>(static_cast<int>(r[i + 3])), c, c, nb, nb);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            pv[e] = ex2_approx(y[e]);
+            if (MASK && col0 + i + e >= n_valid) pv[e] = 0.f;
+        }
+        fadd2(acc[0], acc[1], acc[0], acc[1], pv[0], pv[1]);
+        fadd2(acc[2], acc[3], acc[2], acc[3], pv[2], pv[3]);
+        w[i / 4] = cvt_e4m3x2(pv[0], pv[1]) | (cvt_e4m3x2(pv[2], pv[3]) << 16);
+    }
+}
+
+// Row `row` of a 128-byte-swizzled K-major tile (8-row atoms of 1024 bytes):
+// 16-byte chunk c of the row lives at row*128 + ((c ^ (row & 7)) * 16).
+__device__ __forceinline__ void store_p_row(uint32_t tile, int row, const uint32_t (&w)[32]) {
+    const uint32_t rbase = tile + row * 128;
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+        st_shared_v4(rbase + ((c ^ (row & 7)) << 4), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);
@@ -109,7 +181,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     uint8_t *sQ = base;
     uint8_t *sK = base + 2 * C::Q_BYTES;
     uint8_t *sV = sK + C::STAGES * C::K_BYTES;
-    Ctl<D> *ctl = reinterpret_cast<Ctl<D> *>(sV + C::STAGES * C::V_BYTES);
+    uint8_t *sP = sV + C::STAGES * C::V_BYTES;  // [tile][buffer] P tiles
+    Ctl<D> *ctl = reinterpret_cast<Ctl<D> *>(sP + 4 * C::P_BYTES);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = EXPORT_S ? p.bh0 : static_cast<int>(blockIdx.y);
@@ -125,8 +198,11 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         }
         for (int t = 0; t < 2; ++t) {
             mbar_init(&ctl->s_full[t], 1);
-            mbar_init(&ctl->p_ready[t], 128);
+            mbar_init(&ctl->s_free[t], 4);      // one arrival per softmax warp
+            mbar_init(&ctl->p_ready[t][0], 4);
+            mbar_init(&ctl->p_ready[t][1], 4);
             mbar_init(&ctl->o_done[t], 1);
+            mbar_init(&ctl->o_final[t], 1);
         }
         mbar_init(&ctl->drain, 1);
         ctl->abort.flag = 0;
@@ -147,6 +223,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
+    if (warp >= 8) regs_decrease<C::OTHER_REGS>();
     if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -157,7 +234,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             for (int j = 0; j < nkv; ++j) {
                 const int s = j % C::STAGES;
                 if (j >= C::STAGES &&
-                    !wait_one(&ctl->kv_empty[s], ((j / C::STAGES) - 1) & 1, p.err, &ctl->abort))
+                    !wait_one(&ctl->kv_empty[s], ((j / C::STAGES) - 1) & 1, p.err, &ctl->abort, false, 1))
                     break;
                 mbar_arrive_expect_tx(&ctl->kv_full[s], EXPORT_S ? C::K_BYTES : C::K_BYTES + C::V_BYTES);
                 tma_load_3d(sK + s * C::K_BYTES, &tm_k, &ctl->kv_full[s], 0, (kv0 + j) * C::BN, bh);
@@ -166,37 +243,37 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 issued = j + 1;
             }
             // every copy started here lands before the CTA may exit
-            wait_one(&ctl->q_full, 0, p.err, &ctl->abort, true);
+            wait_one(&ctl->q_full, 0, p.err, &ctl->abort, true, 2);
             for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
-                wait_one(&ctl->kv_full[j % C::STAGES], (j / C::STAGES) & 1, p.err, &ctl->abort, true);
+                wait_one(&ctl->kv_full[j % C::STAGES], (j / C::STAGES) & 1, p.err, &ctl->abort, true, 3);
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA issue
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_i8_s32(128, C::BN);
             const uint32_t idesc_pv = idesc_e4m3_f32(128, D);
-            const uint32_t q_addr[2] = {smem_u32(sQ), smem_u32(sQ) + C::Q_BYTES};
+            const uint32_t q_addr = smem_u32(sQ);
+            const uint32_t p_addr = smem_u32(sP);
             auto issue_qk = [&](int t, int s) {
                 const uint32_t kb = smem_u32(sK + s * C::K_BYTES);
-                const uint32_t dt = tmem + (t ? C::T_S1 : C::T_S0);
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
-                    mma_i8_ss(dt, smem_desc_kmajor(q_addr[t] + kk * 32, D), smem_desc_kmajor(kb + kk * 32, D),
-                              idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_i8_ss(tmem + t * 128, smem_desc_kmajor(q_addr + t * C::Q_BYTES + kk * 32, D),
+                              smem_desc_kmajor(kb + kk * 32, D), idesc_qk, kk > 0 ? 1u : 0u);
                 tc_commit(&ctl->s_full[t]);
             };
             auto issue_pv = [&](int t, int s, int j) {
                 const uint32_t vb = smem_u32(sV + s * C::V_BYTES);
-                const uint32_t dt = tmem + (t ? C::T_O1 : C::T_O0);
-                const uint32_t at = tmem + (t ? C::T_S1 : C::T_S0);
+                const uint32_t pb = p_addr + (2 * t + (j & 1)) * C::P_BYTES;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 32; ++kk)
-                    mma_f8_ts(dt, at + kk * 8, smem_desc_kmajor(vb + kk * 32, C::BN), idesc_pv,
-                              (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_f8_ss(tmem + C::T_O + t * D, smem_desc_kmajor(pb + kk * 32, C::BN),
+                              smem_desc_kmajor(vb + kk * 32, C::BN), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->o_done[t]);
+                if (j == nkv - 1) tc_commit(&ctl->o_final[t]);
             };
-            bool ok = wait_one(&ctl->q_full, 0, p.err, &ctl->abort) &&
-                      wait_one(&ctl->kv_full[0], 0, p.err, &ctl->abort);
+            bool ok = wait_one(&ctl->q_full, 0, p.err, &ctl->abort, false, 4) &&
+                      wait_one(&ctl->kv_full[0], 0, p.err, &ctl->abort, false, 5);
             if (ok) {
                 tc_fence_after();
                 issue_qk(0, 0);
@@ -204,42 +281,57 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             }
             for (int j = 0; ok && j < nkv; ++j) {
                 const int s = j % C::STAGES;
-                if (!(ok = wait_one(&ctl->p_ready[0], j & 1, p.err, &ctl->abort))) break;
-                tc_fence_after();
-                if (!EXPORT_S) issue_pv(0, s, j);
                 if (j + 1 < nkv) {
-                    const int s2 = (j + 1) % C::STAGES;
-                    if (!(ok = wait_one(&ctl->kv_full[s2], ((j + 1) / C::STAGES) & 1, p.err, &ctl->abort))) break;
-                    tc_fence_after();
-                    issue_qk(0, s2);
+                    const int s1 = (j + 1) % C::STAGES;
+                    if (!(ok = wait_one(&ctl->kv_full[s1], ((j + 1) / C::STAGES) & 1, p.err, &ctl->abort, false, 6)))
+                        break;
+                    for (int t = 0; ok && t < 2; ++t) {
+                        if (!(ok = wait_one(&ctl->s_free[t], j & 1, p.err, &ctl->abort, false, 7))) break;
+                        tc_fence_after();
+                        issue_qk(t, s1);  // the tile's softmax holds S(j) in registers already
+                    }
+                } else {
+                    for (int t = 0; ok && t < 2; ++t)
+                        ok = wait_one(&ctl->s_free[t], j & 1, p.err, &ctl->abort, false, 7);
                 }
-                if (!(ok = wait_one(&ctl->p_ready[1], j & 1, p.err, &ctl->abort))) break;
-                tc_fence_after();
-                if (!EXPORT_S) issue_pv(1, s, j);
-                tc_commit(&ctl->kv_empty[s]);
-                if (j + 1 < nkv) issue_qk(1, (j + 1) % C::STAGES);
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (!(ok = wait_one(&ctl->p_ready[t][j & 1], (j >> 1) & 1, p.err, &ctl->abort, false, 8))) break;
+                    tc_fence_after();
+                    if (!EXPORT_S) issue_pv(t, s, j);
+                }
+                if (ok) tc_commit(&ctl->kv_empty[s]);
             }
             // all MMAs issued here finish before tensor memory is released
             tc_commit(&ctl->drain);
-            wait_one(&ctl->drain, 0, p.err, &ctl->abort, true);
+            wait_one(&ctl->drain, 0, p.err, &ctl->abort, true, 9);
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
+        regs_increase<C::SOFTMAX_REGS>();
         const int t = warp >> 2;         // Q tile of this warpgroup
         const int wq = warp & 3;         // tensor-memory lane quarter
-        const int row_in_tile = wq * 32 + lane;
+        const int row = wq * 32 + lane;  // query row within the tile
         const int qt = qt0 + t;
-        const int row = qt * C::BM + row_in_tile;
+        const int grow = qt * C::BM + row;
         const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-        const uint32_t tS = tmem + lane_off + (t ? C::T_S1 : C::T_S0);
-        const uint32_t tO = tmem + lane_off + (t ? C::T_O1 : C::T_O0);
+        const uint32_t tS = tmem + lane_off + t * 128;
+        const uint32_t tO = tmem + lane_off + C::T_O + t * D;
+        const uint32_t pbase = smem_u32(sP) + 2 * t * C::P_BYTES;
         const float sq = qt < p.nqb ? p.q_scale[(int64_t)bh * p.nqb + qt] : 0.f;
         const float cq = sq * p.s_l2;
         const float kLog2_448 = 8.807354922057604f;
+        const float *ksc = p.k_scale + (int64_t)bh * p.nkb + 2 * kv0;
         float m = -INFINITY, l = 0.f;
+        float ks_next0 = EXPORT_S ? 0.f : __ldg(ksc), ks_next1 = EXPORT_S ? 0.f : __ldg(ksc + 1);
         bool ok = true;
-        for (int j = 0; j < nkv; ++j) {
-            if (!(ok = wait_warp(&ctl->s_full[t], j & 1, p.err, &ctl->abort))) break;
+        for (int j = 0; ok && j < nkv; ++j) {
+            // this step's two K-block scales were fetched one step ahead
+            const float ks0 = ks_next0, ks1 = ks_next1;
+            if (!EXPORT_S && j + 1 < nkv) {
+                ks_next0 = __ldg(ksc + 2 * (j + 1));
+                ks_next1 = __ldg(ksc + 2 * (j + 1) + 1);
+            }
+            if (!(ok = wait_warp(&ctl->s_full[t], j & 1, p.err, &ctl->abort, 10 + t))) break;
             tc_fence_after();
             uint32_t ra[32], rb[32], rc[32], rd[32];
             tmem_ld_32x32b_x32(tS + 0, ra);
@@ -250,10 +342,13 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             tmem_wait_ld_x32(rb);
             tmem_wait_ld_x32(rc);
             tmem_wait_ld_x32(rd);
-            uint32_t pk[32];
+            // S(j) is in registers: the tensor core may overwrite it with S(j+1)
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->s_free[t]);
             if (EXPORT_S) {
                 if (t == 0) {
-                    int32_t *dst = p.s_export + row_in_tile * C::BN;
+                    int32_t *dst = p.s_export + row * C::BN;
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         dst[i] = static_cast<int32_t>(ra[i]);
@@ -262,62 +357,48 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                         dst[96 + i] = static_cast<int32_t>(rd[i]);
                     }
                 }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) pk[i] = 0;
             } else {
-                const int kvt = kv0 + j;
-                const int kv_valid = min(C::BN, p.N - kvt * C::BN);
-                const float c0 = cq * p.k_scale[(int64_t)bh * p.nkb + 2 * kvt];
-                const float c1 = cq * p.k_scale[(int64_t)bh * p.nkb + 2 * kvt + 1];
-                if (kv_valid < C::BN) {
+                const int n_valid = min(C::BN, p.N - (kv0 + j) * C::BN);
+                const float c0 = cq * ks0, c1 = cq * ks1;
+                float x0, x1;
+                if (n_valid == C::BN) {
+                    x0 = static_cast<float>(row_max64<false>(ra, rb, 0, n_valid)) * c0;
+                    x1 = static_cast<float>(row_max64<false>(rc, rd, 64, n_valid)) * c1;
+                } else {
                     // ragged last step: keys at or past N take no part
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        if (i >= kv_valid) ra[i] = static_cast<uint32_t>(INT_MIN);
-                        if (32 + i >= kv_valid) rb[i] = static_cast<uint32_t>(INT_MIN);
-                        if (64 + i >= kv_valid) rc[i] = static_cast<uint32_t>(INT_MIN);
-                        if (96 + i >= kv_valid) rd[i] = static_cast<uint32_t>(INT_MIN);
-                    }
+                    const int mx0 = row_max64<true>(ra, rb, 0, n_valid);
+                    const int mx1 = row_max64<true>(rc, rd, 64, n_valid);
+                    x0 = mx0 == INT_MIN ? -INFINITY : static_cast<float>(mx0) * c0;
+                    x1 = mx1 == INT_MIN ? -INFINITY : static_cast<float>(mx1) * c1;
                 }
-                int mx0 = INT_MIN, mx1 = INT_MIN;
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    mx0 = max(mx0, max(static_cast<int>(ra[i]), static_cast<int>(rb[i])));
-                    mx1 = max(mx1, max(static_cast<int>(rc[i]), static_cast<int>(rd[i])));
-                }
-                const float x0 = mx0 == INT_MIN ? -INFINITY : static_cast<float>(mx0) * c0;
-                const float x1 = mx1 == INT_MIN ? -INFINITY : static_cast<float>(mx1) * c1;
                 const float m_new = fmaxf(m, ceilf(fmaxf(x0, x1)));
                 const float alpha = (m == -INFINITY) ? 0.f : exp2_int(m - m_new);
                 const float nb = kLog2_448 - m_new;
-                float sum = 0.f;
-                auto emit = [&](const uint32_t (&r)[32], float cc, int col0, uint32_t *dst) {
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        float pv[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int sv = static_cast<int>(r[i + e]);
-                            float pe = ex2_approx(fmaf(static_cast<float>(sv), cc, nb));
-                            if (col0 + i + e >= kv_valid) pe = 0.f;
-                            pv[e] = pe;
-                        }
-                        sum += (pv[0] + pv[1]) + (pv[2] + pv[3]);
-                        dst[i / 4] = cvt_e4m3x2(pv[0], pv[1]) | (cvt_e4m3x2(pv[2], pv[3]) << 16);
-                    }
-                };
-                emit(ra, c0, 0, pk + 0);
-                emit(rb, c0, 32, pk + 8);
-                emit(rc, c1, 64, pk + 16);
-                emit(rd, c1, 96, pk + 24);
-                l = l * alpha + sum;
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+                uint32_t w[32];
+                if (n_valid == C::BN) {
+                    p_pack32<false>(ra, c0, nb, 0, n_valid, acc, w + 0);
+                    p_pack32<false>(rb, c0, nb, 32, n_valid, acc, w + 8);
+                    p_pack32<false>(rc, c1, nb, 64, n_valid, acc, w + 16);
+                    p_pack32<false>(rd, c1, nb, 96, n_valid, acc, w + 24);
+                } else {
+                    p_pack32<true>(ra, c0, nb, 0, n_valid, acc, w + 0);
+                    p_pack32<true>(rb, c0, nb, 32, n_valid, acc, w + 8);
+                    p_pack32<true>(rc, c1, nb, 64, n_valid, acc, w + 16);
+                    p_pack32<true>(rd, c1, nb, 96, n_valid, acc, w + 24);
+                }
+                l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                // P buffer j%2 was last read by PV(j-2), which finished before S(j)
+                // did (the MMAs run in order), so it can be overwritten now
+                store_p_row(pbase + (j & 1) * C::P_BYTES, row, w);
+                fence_proxy_async_smem();  // make the stores visible to the tensor core
                 const bool need = (j > 0) && (m_new > m);
                 m = m_new;
-                tmem_st_32x32b_x32(tS + 0, pk);
-                tmem_wait_st();
                 if (__any_sync(0xffffffffu, need)) {
-                    // O must hold step j-1's product before it is rescaled
-                    if (!(ok = wait_warp(&ctl->o_done[t], (j - 1) & 1, p.err, &ctl->abort))) break;
+                    // O must hold step j-1's product before it is rescaled; S(j)
+                    // arriving proves PV(j-2) finished, so this barrier is at most
+                    // one phase behind
+                    if (!(ok = wait_warp(&ctl->o_done[t], (j - 1) & 1, p.err, &ctl->abort, 12))) break;
                     tc_fence_after();
                     const float a = need ? alpha : 1.f;
 #pragma unroll 1
@@ -332,37 +413,32 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     tmem_wait_st();
                 }
             }
-            if (EXPORT_S) {
-                tmem_st_32x32b_x32(tS + 0, pk);
-                tmem_wait_st();
-            }
             tc_fence_before();
-            mbar_arrive(&ctl->p_ready[t]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->p_ready[t][j & 1]);
         }
-        if (ok && !EXPORT_S) {
-            if (wait_warp(&ctl->o_done[t], (nkv - 1) & 1, p.err, &ctl->abort)) {
-                tc_fence_after();
-                const float inv_l = 1.f / l;
-                uint16_t *orow = p.out + (int64_t)(bh / p.H) * p.osb + (int64_t)(bh % p.H) * p.osh +
-                                 (int64_t)row * p.osn;
+        if (ok && !EXPORT_S && wait_warp(&ctl->o_final[t], 0, p.err, &ctl->abort, 13)) {
+            tc_fence_after();
+            const float inv_l = 1.f / l;
+            uint16_t *orow = p.out + (int64_t)(bh / p.H) * p.osb + (int64_t)(bh % p.H) * p.osh +
+                             (int64_t)grow * p.osn;
 #pragma unroll 1
-                for (int cc = 0; cc < D / 32; ++cc) {
-                    uint32_t o[32];
-                    tmem_ld_32x32b_x32(tO + cc * 32, o);
-                    tmem_wait_ld_x32(o);
-                    uint32_t w[16];
+            for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[32];
+                tmem_ld_32x32b_x32(tO + cc * 32, o);
+                tmem_wait_ld_x32(o);
+                uint32_t w[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int c = cc * 32 + 2 * i;
-                        w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * ctl->v_scale[c] * inv_l,
-                                           __uint_as_float(o[2 * i + 1]) * ctl->v_scale[c + 1] * inv_l);
-                    }
-                    if (row < p.N) {
-                        uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
+                for (int i = 0; i < 16; ++i) {
+                    const int cidx = cc * 32 + 2 * i;
+                    w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * ctl->v_scale[cidx] * inv_l,
+                                       __uint_as_float(o[2 * i + 1]) * ctl->v_scale[cidx + 1] * inv_l);
+                }
+                if (grow < p.N) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
-                    }
+                    for (int i = 0; i < 4; ++i)
+                        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
                 }
             }
         }
@@ -432,7 +508,7 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if ((e = make_map(&tq, q_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BM)) != cudaSuccess) return e;
     if ((e = make_map(&tk, k_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) return e;
     if (EXPORT_S) {
-        tv = tk;
+        tv = tk;  // not read
     } else if ((e = make_map(&tv, v_t8, n_pad, D, s.BH(), n_pad, (uint64_t)n_pad * D, C::BN, D)) != cudaSuccess) {
         return e;
     }
@@ -441,6 +517,11 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if (!p.err) return cudaErrorSymbolNotFound;
     const int smem = smem_bytes<D>();
     auto kern = k_attn<D, EXPORT_S>;
+    // The setmaxnreg split assumes the kernel is launched with LAUNCH_REGS per
+    // thread; with fewer the increases could never be satisfied.
+    cudaFuncAttributes fa;
+    if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
+    if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
     kern<<<grid, C::THREADS, smem, st>>>(tq, tk, tv, p);
     return cudaGetLastError();

@@ -10,7 +10,8 @@
 
 namespace sage {
 
-// Bit set in the device error word when a bounded wait gave up.
+// Bit set in the device error word when a bounded wait gave up; the wait's
+// site (which barrier) is recorded as bit (8 + site).
 constexpr unsigned kErrTimeout = 1u;
 
 // A wait longer than this many SM clocks (~1 s at 2 GHz) is treated as a hang.
@@ -54,8 +55,8 @@ struct AbortState {
     int flag;  // set (to 1) in shared memory by the first thread that gives up
 };
 
-__device__ __forceinline__ void record_timeout(unsigned *err_word, AbortState *st) {
-    atomicOr(err_word, kErrTimeout);
+__device__ __forceinline__ void record_timeout(unsigned *err_word, AbortState *st, int site = 0) {
+    atomicOr(err_word, kErrTimeout | (1u << (8 + (site & 15))));
     *reinterpret_cast<volatile int *>(&st->flag) = 1;
 }
 
@@ -63,12 +64,12 @@ __device__ __forceinline__ void record_timeout(unsigned *err_word, AbortState *s
 // Returns false (after recording the timeout) if it gave up or if another
 // thread of the CTA already gave up (unless ignore_abort is set).
 __device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, unsigned *err_word,
-                                         AbortState *st, bool ignore_abort = false) {
+                                         AbortState *st, bool ignore_abort = false, int site = 0) {
     long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (!ignore_abort && *reinterpret_cast<volatile int *>(&st->flag)) return false;
         if (clock64() - t0 > kWaitLimitClocks) {
-            record_timeout(err_word, st);
+            record_timeout(err_word, st, site);
             return false;
         }
     }
@@ -78,7 +79,7 @@ __device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, unsigne
 // Warp-uniform bounded wait: every lane of the warp returns the same value,
 // so .sync.aligned instructions that follow stay convergent.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, unsigned *err_word,
-                                          AbortState *st) {
+                                          AbortState *st, int site = 0) {
     long long t0 = clock64();
     while (true) {
         bool ok = mbar_try_wait(bar, parity);
@@ -86,7 +87,10 @@ __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, unsign
         bool give_up = *reinterpret_cast<volatile int *>(&st->flag) != 0 ||
                        (clock64() - t0 > kWaitLimitClocks);
         if (__any_sync(0xffffffffu, give_up)) {
-            if ((threadIdx.x & 31) == 0) record_timeout(err_word, st);
+            if ((threadIdx.x & 31) == 0 && !*reinterpret_cast<volatile int *>(&st->flag))
+                record_timeout(err_word, st, site);
+            else if ((threadIdx.x & 31) == 0)
+                record_timeout(err_word, st, 15);  // gave up because another wait did
             __syncwarp();
             return false;
         }
@@ -107,6 +111,17 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const CUtensorMap *m
         " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
         : "memory");
+}
+
+// Per-warpgroup register reallocation (every warp of a warpgroup executes the
+// same one).  The increases draw on the registers the block was launched with.
+template <uint32_t N>
+__device__ __forceinline__ void regs_increase() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_decrease() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
 // ------------------------------------------------------------------- tcgen05
@@ -152,6 +167,21 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+// D(tmem) (+)= A(smem) * B(smem)^T, 8-bit float inputs (types from idesc), fp32 accumulate.
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// 16-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -217,12 +247,37 @@ __device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_
                  : "memory");
 }
 
+__device__ __forceinline__ void tmem_st_32x32b_x8(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :
+                 : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 // Two fp32 -> two e4m3 (round to nearest even, saturate to +-448) packed in
 // 16 bits: `lo` in bits 0-7, `hi` in bits 8-15.
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
+}
+
+// Packed fp32 pair arithmetic of sm_100 (one instruction, two IEEE results,
+// each rounded to nearest even exactly as the scalar form would be).
+__device__ __forceinline__ void fadd2(float &d0, float &d1, float a0, float a1, float b0, float b1) {
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
