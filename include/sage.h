@@ -142,14 +142,13 @@ sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t q_stride[4
 /*
  * sage_quant_v -- V to FP8 e4m3 with one scale per (b,h,channel) ([H3] "FP8 for
  * PV"; reading C7):  amax_c = max_n |V|;  v_scale = amax_c/448;
- * v_t8[b,h,c,n] = e4m3_rn_satfinite(V * (448/amax_c)).
- * Outputs: v_t8 uint8 (e4m3 bits) [B,H,d,N_pad] -- channel-major, i.e. V
- * transposed so that the P.V operand is K-major; v_scale float [B,H,d].
- * workspace as for sage_quant_qk.
+ * v_e4m3[b,h,n,c] = e4m3_rn_satfinite(V * (448/amax_c)).
+ * Outputs: v_e4m3 uint8 (e4m3 bits) [B,H,N_pad,d], token-major like the int8
+ * codes; v_scale float [B,H,d].  workspace as for sage_quant_qk.
  */
 sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4],
                            int B, int H, int N, int d,
-                           uint8_t *v_t8, float *v_scale,
+                           uint8_t *v_e4m3, float *v_scale,
                            void *workspace, size_t workspace_bytes,
                            sage_stream_t stream);
 
@@ -165,7 +164,7 @@ sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4],
  */
 sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale,
                                   const int8_t *k_i8, const float *k_scale,
-                                  const uint8_t *v_t8, const float *v_scale,
+                                  const uint8_t *v_e4m3, const float *v_scale,
                                   void *out, const int64_t o_stride[4],
                                   int B, int H, int N, int d, float sm_scale,
                                   sage_stream_t stream);

@@ -156,19 +156,19 @@ def sage_quant_qk_noalloc(q, k, out=None, stream=None):
 
 
 def sage_quant_v(v, workspace=None, stream=None):
-    """V -> e4m3 with per-channel scales.  Returns (v_t8 uint8 [B,H,d,N_pad], v_scale [B,H,d])."""
+    """V -> e4m3 with per-channel scales.  Returns (v_e4m3 uint8 [B,H,N_pad,d], v_scale [B,H,d])."""
     _check_qkv(v)
     B, H, N, d = v.shape
     dev = v.device
-    v_t8 = torch.empty(B, H, d, n_pad(N), dtype=torch.uint8, device=dev)
+    v_e4m3 = torch.empty(B, H, n_pad(N), d, dtype=torch.uint8, device=dev)
     v_scale = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _raise(lib().sage_quant_v(_ptr(v), _strides(v), B, H, N, d, _ptr(v_t8), _ptr(v_scale), _ptr(workspace),
+    _raise(lib().sage_quant_v(_ptr(v), _strides(v), B, H, N, d, _ptr(v_e4m3), _ptr(v_scale), _ptr(workspace),
                               ws_bytes, _stream(stream, dev)))
-    return v_t8, v_scale
+    return v_e4m3, v_scale
 
 
-def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_t8, v_scale, N: int, sm_scale=None, out=None, stream=None):
+def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, N: int, sm_scale=None, out=None, stream=None):
     """The fused attention kernel on existing codes; returns bf16 [B,H,N,d]."""
     B, H, _, d = q_i8.shape
     dev = q_i8.device
@@ -176,10 +176,10 @@ def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_t8, v_scale, N: int, sm_
         sm_scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
-    for t in (q_i8, q_scale, k_i8, k_scale, v_t8, v_scale):
+    for t in (q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale):
         if not t.is_contiguous():
             raise ValueError("code and scale tensors must be contiguous")
-    _raise(lib().sage_attn_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_t8),
+    _raise(lib().sage_attn_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_e4m3),
                                      _ptr(v_scale), _ptr(out), _strides(out), B, H, N, d,
                                      ctypes.c_float(sm_scale), _stream(stream, dev)))
     return out

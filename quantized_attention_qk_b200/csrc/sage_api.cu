@@ -134,7 +134,7 @@ Codes carve_codes(void *base, const Shape &s) {
     Codes c;
     c.q_i8 = reinterpret_cast<int8_t *>(p);
     c.k_i8 = reinterpret_cast<int8_t *>(p + codes);
-    c.v_t8 = reinterpret_cast<uint8_t *>(p + 2 * codes);
+    c.v_e4m3 = reinterpret_cast<uint8_t *>(p + 2 * codes);
     p += 3 * codes;
     c.q_scale = reinterpret_cast<float *>(p);
     p += up((size_t)s.BH() * s.n_qblocks() * 4);
@@ -212,11 +212,12 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4], const
     return SAGE_OK;
 }
 
-sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B, int H, int N, int d, uint8_t *v_t8,
-                           float *v_scale, void *workspace, size_t workspace_bytes, sage_stream_t stream) {
+sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B, int H, int N, int d,
+                           uint8_t *v_e4m3, float *v_scale, void *workspace, size_t workspace_bytes,
+                           sage_stream_t stream) {
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_view(v_bf16, v_stride, "v")) ||
-        (r = check_dev(v_t8, "v_t8", 16)) || (r = check_dev(v_scale, "v_scale", 4)))
+        (r = check_dev(v_e4m3, "v_e4m3", 16)) || (r = check_dev(v_scale, "v_scale", 4)))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -225,7 +226,7 @@ sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B,
     const StatsWs ws = carve_stats_ws(scr.ptr, s);
     const Src vs = src(v_bf16, v_stride);
     Codes c{};
-    c.v_t8 = v_t8;
+    c.v_e4m3 = v_e4m3;
     c.v_scale = v_scale;
     cudaError_t e = launch_stats(s, nullptr, &vs, ws, nullptr, v_scale, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
@@ -240,11 +241,11 @@ static sage_status_t check_scale(float sm_scale) {
 }
 
 sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8, const float *k_scale,
-                                  const uint8_t *v_t8, const float *v_scale, void *out, const int64_t o_stride[4],
+                                  const uint8_t *v_e4m3, const float *v_scale, void *out, const int64_t o_stride[4],
                                   int B, int H, int N, int d, float sm_scale, sage_stream_t stream) {
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_dev(q_i8, "q_i8", 16)) ||
-        (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(v_t8, "v_t8", 16)) ||
+        (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(v_e4m3, "v_e4m3", 16)) ||
         (r = check_dev(q_scale, "q_scale", 4)) || (r = check_dev(k_scale, "k_scale", 4)) ||
         (r = check_dev(v_scale, "v_scale", 4)) || (r = check_view(out, o_stride, "out")))
         return r;
@@ -254,7 +255,7 @@ sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale, cons
     c.q_scale = const_cast<float *>(q_scale);
     c.k_i8 = const_cast<int8_t *>(k_i8);
     c.k_scale = const_cast<float *>(k_scale);
-    c.v_t8 = const_cast<uint8_t *>(v_t8);
+    c.v_e4m3 = const_cast<uint8_t *>(v_e4m3);
     c.v_scale = const_cast<float *>(v_scale);
     cudaError_t e = launch_attention(s, c, dst(out, o_stride), sm_scale, reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "attention kernel");

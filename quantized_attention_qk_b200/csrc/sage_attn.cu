@@ -9,11 +9,13 @@
 // Warp roles (384 threads, three warpgroups):
 //   warpgroup t (warps 4t..4t+3), t = 0, 1: softmax of Q tile t, one query row
 //              per thread; the two warpgroups run independently of each other
-//   warp 8     TMA producer: both Q tiles once, then a ring of (K, V^T) stages
+//   warp 8     TMA producer: both Q tiles once, then a ring of (K, V) stages
 //   warp 9     tensor-memory allocator and single-thread tcgen05.mma issuer
 //   warps 10-11 idle
 // After set-up the softmax warpgroups raise their register limit to 224 and
 // warpgroup 2 lowers its own to 48 (setmaxnreg).
+// V tiles are loaded token-major (key rows of d channels) and fed to the P.V MMA
+// as an MN-major operand.
 // Tensor memory (512 columns x 128 lanes): S0, S1 (int32, 128 columns each) at
 // [0,256), O0, O1 (fp32, d columns each) from 256.
 // P (e4m3) goes to shared memory, two buffers per tile, in the 128-byte-swizzled
@@ -54,7 +56,7 @@ struct Cfg {
     static constexpr int STAGES = 3;
     static constexpr int Q_BYTES = BM * D;
     static constexpr int K_BYTES = BN * D;
-    static constexpr int V_BYTES = D * BN;
+    static constexpr int V_BYTES = BN * D;          // V tile: BN key rows of d e4m3 channels
     static constexpr int P_BYTES = BM * BN;        // one P buffer (e4m3)
     static constexpr int TILE_BYTES = 2 * Q_BYTES + STAGES * (K_BYTES + V_BYTES) + 4 * P_BYTES;
     static constexpr uint32_t T_O = 256;           // O of tile t at 256 + d t
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 mbar_arrive_expect_tx(&ctl->kv_full[s], EXPORT_S ? C::K_BYTES : C::K_BYTES + C::V_BYTES);
                 tma_load_3d(sK + s * C::K_BYTES, &tm_k, &ctl->kv_full[s], 0, (kv0 + j) * C::BN, bh);
                 if (!EXPORT_S)
-                    tma_load_3d(sV + s * C::V_BYTES, &tm_v, &ctl->kv_full[s], (kv0 + j) * C::BN, 0, bh);
+                    tma_load_3d(sV + s * C::V_BYTES, &tm_v, &ctl->kv_full[s], 0, (kv0 + j) * C::BN, bh);
                 issued = j + 1;
             }
             // every copy started here lands before the CTA may exit
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         // ----------------------------------------------------------- MMA issue
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_i8_s32(128, C::BN);
-            const uint32_t idesc_pv = idesc_e4m3_f32(128, D);
+            const uint32_t idesc_pv = idesc_e4m3_f32_bmn(128, D);
             const uint32_t q_addr = smem_u32(sQ);
             const uint32_t p_addr = smem_u32(sP);
             auto issue_qk = [&](int t, int s) {
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 32; ++kk)
                     mma_f8_ss(tmem + C::T_O + t * D, smem_desc_kmajor(pb + kk * 32, C::BN),
-                              smem_desc_kmajor(vb + kk * 32, C::BN), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                              smem_desc_mnmajor(vb + kk * 32 * D, D), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->o_done[t]);
                 if (j == nkv - 1) tc_commit(&ctl->o_final[t]);
             };
@@ -499,7 +501,7 @@ unsigned *device_error_ptr() {
 }
 
 template <int D, bool EXPORT_S>
-cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_t8,
+cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
                           const AttnParams &p0, dim3 grid, cudaStream_t st) {
     using C = Cfg<D>;
     const int n_pad = s.n_pad();
@@ -509,7 +511,7 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if ((e = make_map(&tk, k_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) return e;
     if (EXPORT_S) {
         tv = tk;  // not read
-    } else if ((e = make_map(&tv, v_t8, n_pad, D, s.BH(), n_pad, (uint64_t)n_pad * D, C::BN, D)) != cudaSuccess) {
+    } else if ((e = make_map(&tv, v_e4m3, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) {
         return e;
     }
     AttnParams p = p0;
@@ -544,8 +546,8 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
     p.nkb = s.n_kblocks();
     p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
-    return s.d == 128 ? launch_attn_d<128, false>(s, c.q_i8, c.k_i8, c.v_t8, p, grid, st)
-                      : launch_attn_d<64, false>(s, c.q_i8, c.k_i8, c.v_t8, p, grid, st);
+    return s.d == 128 ? launch_attn_d<128, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
+                      : launch_attn_d<64, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
 }
 
 cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,

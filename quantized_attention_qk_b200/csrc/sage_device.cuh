@@ -198,6 +198,17 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t ro
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (sbo << 32) | (1ull << 46) | (layout << 61);
 }
 
+// Shared-memory matrix descriptor for an MN-major 8-bit operand tile written by
+// TMA with a 128-byte (layout 2) or 64-byte (layout 4) swizzle: the MN extent
+// (row_bytes elements) is contiguous within a row and the operand's K index
+// runs over rows; 8-row groups are 8*row_bytes apart (stride offset).  The MN
+// extent equals one swizzle atom, so the leading offset is not used.
+__device__ __forceinline__ uint64_t smem_desc_mnmajor(uint32_t saddr, uint32_t row_bytes) {
+    const uint64_t layout = (row_bytes == 128) ? 2ull : 4ull;
+    const uint64_t sbo = (8u * row_bytes) >> 4;
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (sbo << 32) | (1ull << 46) | (layout << 61);
+}
+
 // Instruction descriptors (kind::i8 and kind::f8f6f4 share the layout):
 // [4,6) D type (1 f32, 2 s32), [7,10) A type, [10,13) B type, [15] A MN-major,
 // [16] B MN-major, [17,23) N>>3, [24,29) M>>4.
@@ -206,6 +217,10 @@ __host__ __device__ constexpr uint32_t idesc_i8_s32(uint32_t M, uint32_t N) {
 }
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// The same with an MN-major B operand (bit 16).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_bmn(uint32_t M, uint32_t N) {
+    return idesc_e4m3_f32(M, N) | (1u << 16);
 }
 
 __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {

@@ -11,7 +11,7 @@ namespace sage {
 constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
 constexpr int kKBlock = 64;        // K tokens per quantization block
 constexpr int kKvTile = 128;       // keys per attention KV tile (two K blocks)
-constexpr int kStatsChunk = 512;   // tokens per CTA of the statistics pass
+constexpr int kStatsCtas = 592;    // statistics pass: aim for 4 CTAs per SM on 148 SMs
 constexpr unsigned kErrTimeoutBit = 1u;  // device error word: a bounded wait gave up
 
 // A bf16 [B,H,N,d] tensor given by base pointer and element strides (c stride 1).
@@ -30,7 +30,15 @@ struct Shape {
     int n_pad() const { return ((N + kQBlock - 1) / kQBlock) * kQBlock; }
     int n_qblocks() const { return n_pad() / kQBlock; }
     int n_kblocks() const { return n_pad() / kKBlock; }
-    int n_chunks() const { return (N + kStatsChunk - 1) / kStatsChunk; }
+    // Statistics pass: each (b,h) is cut into n_chunks() token chunks of
+    // chunk_rows() rows (a multiple of 64), enough CTAs to fill the GPU.
+    int chunk_rows() const {
+        int want = (kStatsCtas + BH() - 1) / BH();
+        int rows = (N + want - 1) / want;
+        rows = (rows + 63) / 64 * 64;
+        return rows < 64 ? 64 : rows;
+    }
+    int n_chunks() const { return (N + chunk_rows() - 1) / chunk_rows(); }
 };
 
 // Scratch of the quantize pass: per-chunk partials and the finished statistics.
@@ -47,7 +55,7 @@ struct Codes {
     float *q_scale;    // [BH][N_pad/128]
     int8_t *k_i8;      // [BH][N_pad][d]
     float *k_scale;    // [BH][N_pad/64]
-    uint8_t *v_t8;     // [BH][d][N_pad]  e4m3 bits
+    uint8_t *v_e4m3;   // [BH][N_pad][d]  e4m3 bits, token-major like the int8 codes
     float *v_scale;    // [BH][d]
 };
 

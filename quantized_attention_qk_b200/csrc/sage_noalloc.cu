@@ -62,8 +62,8 @@ extern "C" sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t
     const Shape s{B, H, N, d};
     const size_t need = stats_ws_bytes(s);
     if (need > kNoAllocScratchBytes) {
-        set_last_error("sage_quant_qk_noalloc: this shape needs %zu bytes of scratch; the built-in scratch "
-                       "holds %zu (B*H*ceil(N/512)*d is too large)",
+        set_last_error("sage_quant_qk_noalloc: this shape needs %zu bytes of scratch "
+                       "(sage_quant_workspace_bytes); the built-in scratch holds %zu",
                        need, kNoAllocScratchBytes);
         return SAGE_ERR_WORKSPACE;
     }

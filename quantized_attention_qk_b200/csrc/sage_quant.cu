@@ -1,18 +1,18 @@
 // sage_quant.cu -- the quantize pass of the quantized attention forward.
 //
 // Three HBM-bound streaming kernels (no tensor cores: there is no contraction):
-//   k_stats_partial  per (b,h, 512-token chunk): sum of K and max |V| per channel
+//   k_stats_partial  per (b,h, token chunk): sum of K and max |V| per channel
 //   k_stats_final    per (b,h): K mean (the smoothing statistic) and 448/amax of V
 //   k_quant          per (b,h, 128-token block): Q block -> INT8, (K - mean) per
-//                    64-token block -> INT8, V -> e4m3 written channel-major.
+//                    64-token block -> INT8, V -> e4m3 (token-major, like the codes
+//                    of Q and K; the attention kernel reads it as an MN-major operand).
 // Pages: "MiniMax H3 接入 SageAttention 实测加速", section 一 (outlier smoothing of
 // QK^T, INT8 QK, FP8 PV).  Block sizes, rounding and scale conventions are the
 // readings C1-C3 and C7 of the design notes:
 //   scale = amax/127 (fp32 IEEE divide), code = rne(x * fp32(127/amax)) in
 //   [-127,127]; V: code = e4m3_rn_satfinite(v * fp32(448/amax_c)).
 // Loads are 16-byte vectors from arbitrary (b,h,n) strides, so a fused-qkv
-// view is read in place; stores are 8-byte (int8 codes) and 16-byte (the
-// transposed e4m3 tile, staged through shared memory) vectors.
+// view is read in place; codes are stored as 8-byte vectors.
 #include <cuda_runtime.h>
 
 #include "sage_internal.h"
@@ -65,8 +65,8 @@ __device__ __forceinline__ uint32_t i8code(float x, float inv) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreads) k_stats_partial(Src k, Src v, int H, int N, int nch, int do_k,
-                                                            int do_v, float *ksum_part, float *vmax_part) {
+__global__ void __launch_bounds__(kThreads) k_stats_partial(Src k, Src v, int H, int N, int nch, int chunk,
+                                                            int do_k, int do_v, float *ksum_part, float *vmax_part) {
     constexpr int VPR = D / 8;             // 16-byte vectors per token row
     constexpr int RPI = kThreads / VPR;    // rows covered per iteration
     __shared__ float red_s[RPI][D];
@@ -74,22 +74,29 @@ __global__ void __launch_bounds__(kThreads) k_stats_partial(Src k, Src v, int H,
     const int bh = blockIdx.y, ch = blockIdx.x;
     const int b = bh / H, h = bh % H;
     const int cv = threadIdx.x % VPR, r0 = threadIdx.x / VPR;
-    const int n0 = ch * kStatsChunk;
-    const int n1 = min(N, n0 + kStatsChunk);
+    const int n0 = ch * chunk;
+    const int n1 = min(N, n0 + chunk);
     float s[8], m[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) { s[e] = 0.f; m[e] = 0.f; }
     const uint16_t *kp = do_k ? k.p + b * k.sb + h * k.sh + cv * 8 : nullptr;
     const uint16_t *vp = do_v ? v.p + b * v.sb + h * v.sh + cv * 8 : nullptr;
-    for (int n = n0 + r0; n < n1; n += RPI) {
-        float f[8];
-        if (do_k) {
-            unpack8(ld_vec(kp + (int64_t)n * k.sn), f);
+    constexpr int U = 4;  // rows in flight per thread and tensor
+    for (int n = n0 + r0; n < n1; n += U * RPI) {
+        uint4 xk[U], xv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int nn = n + u * RPI;
+            xk[u] = (do_k && nn < n1) ? ld_vec(kp + (int64_t)nn * k.sn) : make_uint4(0, 0, 0, 0);
+            xv[u] = (do_v && nn < n1) ? ld_vec(vp + (int64_t)nn * v.sn) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            float f[8];
+            unpack8(xk[u], f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) s[e] += f[e];
-        }
-        if (do_v) {
-            unpack8(ld_vec(vp + (int64_t)n * v.sn), f);
+            unpack8(xv[u], f);
 #pragma unroll
             for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
         }
@@ -135,9 +142,7 @@ __global__ void __launch_bounds__(kThreads) k_quant(Src q, Src k, Src v, int H, 
     constexpr int VPR = D / 8;
     constexpr int RPI = kThreads / VPR;
     constexpr int NI = kQBlock / RPI;    // vectors per thread in one 128-token block
-    constexpr int TS = kQBlock + 16;     // row pitch (bytes) of the transpose tile
     __shared__ float red[16];
-    __shared__ __align__(16) uint8_t tile[DO_V ? D * TS : 16];
     const int blk = blockIdx.x, bh = blockIdx.y;
     const int b = bh / H, h = bh % H;
     const int cv = threadIdx.x % VPR, r0 = threadIdx.x / VPR;
@@ -221,17 +226,18 @@ __global__ void __launch_bounds__(kThreads) k_quant(Src q, Src k, Src v, int H, 
         float inv[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) inv[e] = v_inv[bh * D + cv * 8 + e];
+        uint4 x[NI];
 #pragma unroll
         for (int i = 0; i < NI; ++i) {
-            const int rr = r0 + i * RPI;
-            const int n = row0 + rr;
-            float f[8];
-            if (n < N) {
-                unpack8(ld_vec(vp + (int64_t)n * v.sn), f);
-            } else {
+            const int n = row0 + r0 + i * RPI;
+            x[i] = n < N ? ld_vec(vp + (int64_t)n * v.sn) : make_uint4(0, 0, 0, 0);
+        }
+        uint8_t *dst = c.v_e4m3 + ((int64_t)bh * n_pad + row0) * D + cv * 8;
 #pragma unroll
-                for (int e = 0; e < 8; ++e) f[e] = 0.f;
-            }
+        for (int i = 0; i < NI; ++i) {
+            float f[8];
+            unpack8(x[i], f);
+            uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 8; e += 2) {
                 uint16_t pr;
@@ -239,16 +245,12 @@ __global__ void __launch_bounds__(kThreads) k_quant(Src q, Src k, Src v, int H, 
                 asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
                     : "=h"(pr)
                     : "f"(__fmul_rn(f[e + 1], inv[e + 1])), "f"(__fmul_rn(f[e], inv[e])));
-                tile[(cv * 8 + e) * TS + rr] = static_cast<uint8_t>(pr & 0xff);
-                tile[(cv * 8 + e + 1) * TS + rr] = static_cast<uint8_t>(pr >> 8);
+                w[e / 2] = pr;
             }
-        }
-        __syncthreads();
-        uint8_t *dst = c.v_t8 + (int64_t)bh * D * n_pad + row0;
-        for (int idx = threadIdx.x; idx < D * (kQBlock / 16); idx += kThreads) {
-            const int ch = idx / (kQBlock / 16), part = idx % (kQBlock / 16);
-            *reinterpret_cast<uint4 *>(dst + (int64_t)ch * n_pad + part * 16) =
-                *reinterpret_cast<const uint4 *>(&tile[ch * TS + part * 16]);
+            uint2 o;
+            o.x = w[0] | (w[1] << 16);
+            o.y = w[2] | (w[3] << 16);
+            *reinterpret_cast<uint2 *>(dst + (int64_t)(r0 + i * RPI) * D) = o;
         }
     }
 }
@@ -259,8 +261,8 @@ cudaError_t launch_stats_d(const Shape &s, const Src *k, const Src *v, const Sta
     const int nch = s.n_chunks();
     Src z{nullptr, 0, 0, 0};
     dim3 g1(nch, s.BH());
-    k_stats_partial<D><<<g1, kThreads, 0, st>>>(k ? *k : z, v ? *v : z, s.H, s.N, nch, k != nullptr,
-                                                v != nullptr, ws.ksum_part, ws.vmax_part);
+    k_stats_partial<D><<<g1, kThreads, 0, st>>>(k ? *k : z, v ? *v : z, s.H, s.N, nch, s.chunk_rows(),
+                                                k != nullptr, v != nullptr, ws.ksum_part, ws.vmax_part);
     k_stats_final<D><<<s.BH(), D, 0, st>>>(s.N, nch, k != nullptr, v != nullptr, ws.ksum_part, ws.vmax_part,
                                           ws.k_mean, user_k_mean, ws.v_inv, v_scale);
     return cudaGetLastError();

@@ -63,7 +63,7 @@ def test_quant_codes_match_oracle(name):
     w = WORKLOADS[name]
     (q, k, v), (qd, kd, vd), _ = _inputs(w)
     r = sage.sage_quant_qk(qd, kd)
-    v_t8, v_scale = sage.sage_quant_v(vd)
+    v_e4m3, v_scale = sage.sage_quant_v(vd)
     torch.cuda.synchronize()
     N, npd = w.N, sage.n_pad(w.N)
     heads = [(0, h) for h in range(min(w.H, 3))]
@@ -82,9 +82,9 @@ def test_quant_codes_match_oracle(name):
         dk = gk[:N] - o["k_i8"][0, 0].astype(np.int64)
         assert np.abs(dk).max() <= 1 and (dk != 0).mean() < 1e-3, (np.abs(dk).max(), (dk != 0).mean())
         assert (gk[N:] == 0).all()
-        gv = v_t8[b, h].cpu().numpy()            # [d, N_pad]
-        np.testing.assert_array_equal(gv[:, :N].T, o["v_e4m3"][0, 0])
-        assert (gv[:, N:] == 0).all()
+        gv = v_e4m3[b, h].cpu().numpy()          # [N_pad, d]
+        np.testing.assert_array_equal(gv[:N], o["v_e4m3"][0, 0])
+        assert (gv[N:] == 0).all()
         np.testing.assert_array_equal(v_scale[b, h].cpu().numpy(), o["v_scale"][0, 0])
 
 
@@ -181,11 +181,11 @@ def test_attention_kernel_on_oracle_codes():
 
     q_i8 = torch.from_numpy(pad_rows(o["q_i8"], npd)).to(DEV)
     k_i8 = torch.from_numpy(pad_rows(o["k_i8"], npd)).to(DEV)
-    v_t8 = torch.from_numpy(np.ascontiguousarray(pad_rows(o["v_e4m3"], npd).transpose(0, 1, 3, 2))).to(DEV)
+    v_e4m3 = torch.from_numpy(pad_rows(o["v_e4m3"], npd)).to(DEV)
     qs = np.zeros((1, 2, npd // 128), np.float32); qs[..., :o["q_scale"].shape[-1]] = o["q_scale"]
     ks = np.zeros((1, 2, npd // 64), np.float32); ks[..., :o["k_scale"].shape[-1]] = o["k_scale"]
     out = sage.sage_attn_quantized(q_i8, torch.from_numpy(qs).to(DEV), k_i8, torch.from_numpy(ks).to(DEV),
-                                   v_t8, torch.from_numpy(o["v_scale"]).to(DEV), N, w.sm_scale)
+                                   v_e4m3, torch.from_numpy(o["v_scale"]).to(DEV), N, w.sm_scale)
     torch.cuda.synchronize()
     rows = np.arange(N, dtype=np.int32)
     ref = U.oracle_quant_rows(q, k, v, w.sm_scale, [(0, 0), (0, 1)], rows)

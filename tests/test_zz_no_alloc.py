@@ -25,10 +25,11 @@ def L():
 
 
 def test_noalloc_rejects_a_shape_beyond_its_scratch(L):
-    st = (ctypes.c_int64 * 4)(8 * 65536 * 128, 65536 * 128, 128, 1)
+    st = (ctypes.c_int64 * 4)(128 * 128 * 128, 128 * 128, 128, 1)
     p = ctypes.c_void_p(16 * 4096)
-    # B*H*ceil(N/512)*d*4 bytes of partial sums alone exceed the 4 MiB array
-    rc = L.sage_quant_qk_noalloc(p, st, p, st, 8, 64, 65536, 128, p, p, p, p, None, None)
+    # with B*H = 4096 heads the per-head statistics alone need 8 MB, twice the array
+    assert sage.sage_quant_workspace_bytes(32, 128, 128, 128) > 4 << 20
+    rc = L.sage_quant_qk_noalloc(p, st, p, st, 32, 128, 128, 128, p, p, p, p, None, None)
     assert rc == 3
     assert b"scratch" in L.sage_last_error_message()
 
