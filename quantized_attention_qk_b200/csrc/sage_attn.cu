@@ -12,8 +12,8 @@
 //   warp 8     TMA producer: both Q tiles once, then a ring of (K, V) stages
 //   warp 9     tensor-memory allocator and single-thread tcgen05.mma issuer
 //   warps 10-11 idle
-// After set-up the softmax warpgroups raise their register limit to 224 and
-// warpgroup 2 lowers its own to 48 (setmaxnreg).
+// After set-up the softmax warpgroups raise their register limit to 216 and
+// warpgroup 2 lowers its own to 64 (setmaxnreg).
 // V tiles are loaded token-major (key rows of d channels) and fed to the P.V MMA
 // as an MN-major operand.
 // Tensor memory (512 columns x 128 lanes): S0, S1 (int32, 128 columns each) at
@@ -63,8 +63,8 @@ struct Cfg {
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int THREADS = 384;            // three warpgroups
     static constexpr int LAUNCH_REGS = 168;        // per thread, what 384 threads x 1 block allow
-    static constexpr uint32_t SOFTMAX_REGS = 224;  // warpgroups 0 and 1 after setmaxnreg
-    static constexpr uint32_t OTHER_REGS = 48;     // warpgroup 2 (TMA, MMA, two idle warps)
+    static constexpr uint32_t SOFTMAX_REGS = 216;  // warpgroups 0 and 1 after setmaxnreg
+    static constexpr uint32_t OTHER_REGS = 64;     // warpgroup 2 (TMA, MMA, two idle warps)
     static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= LAUNCH_REGS * THREADS,
                   "register split exceeds the registers the block is launched with");
 };
@@ -134,10 +134,38 @@ __device__ __forceinline__ int row_max64(const uint32_t (&a)[32], const uint32_t
     return max(m0, m1);
 }
 
+// 2^y for two values on the FMA pipe instead of the MUFU unit (16 ex2 per
+// clock per SM, the softmax's limit when both warpgroups exponentiate at once).
+// y = j + f with j the nearest integer (rounded by adding and subtracting
+// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a degree-4 polynomial (Horner),
+// then j is added to the exponent field.  The coefficients minimise the
+// relative error of 2^f on [-1/2, 1/2] (weighted least squares iterated to
+// equal ripple); evaluated in fp32 the relative error stays below 3e-6.  y is
+// clamped at -120 so the exponent cannot underflow (2^-120 is 0 in e4m3).
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float &p0, float &p1) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.9999992847442627f, c1 = 0.6931218504905701f, c2 = 0.240247443318367f,
+                    c3 = 0.05591757968068123f, c4 = 0.009569989517331123f;
+    y0 = fmaxf(y0, -120.f);
+    y1 = fmaxf(y1, -120.f);
+    float t0, t1, j0, j1, f0, f1, q0, q1;
+    fadd2(t0, t1, y0, y1, kRound, kRound);       // integer part in the low mantissa bits
+    fadd2(j0, j1, t0, t1, -kRound, -kRound);     // j as a float
+    ffma2(f0, f1, j0, j1, -1.f, -1.f, y0, y1);   // f = y - j, exact
+    ffma2(q0, q1, c4, c4, f0, f1, c3, c3);
+    ffma2(q0, q1, q0, q1, f0, f1, c2, c2);
+    ffma2(q0, q1, q0, q1, f0, f1, c1, c1);
+    ffma2(q0, q1, q0, q1, f0, f1, c0, c0);
+    // the low bits of t hold j (two's complement); j << 23 lands in the exponent
+    p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(t0) << 23));
+    p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(t1) << 23));
+}
+
 // 448 * 2^(x - m) for 32 scores, x = S * c: y = float(S) * c + (log2 448 - m)
-// (one FMA per pair), p = 2^y on the MUFU unit.  Accumulates the unrounded p
-// into acc and packs the e4m3 codes four per word into w[0..7] (word j holds
-// keys 4j..4j+3, lowest key in the lowest byte).
+// (one FMA per pair), p = 2^y: the MUFU ex2 for six of every eight scores,
+// the polynomial above for the other two.  Accumulates the unrounded p into acc
+// and packs the e4m3 codes four per word into w[0..7] (word j holds keys
+// 4j..4j+3, lowest key in the lowest byte).
 template <bool MASK>
 __device__ __forceinline__ void p_pack32(const uint32_t (&r)[32], float c, float nb, int col0, int n_valid,
                                          float (&acc)[4], uint32_t *w) {
@@ -148,10 +176,18 @@ __device__ __forceinline__ void p_pack32(const uint32_t (&r)[32], float c, float
               c, c, nb, nb);
         ffma2(y[2], y[3], static_cast<float>(static_cast<int>(r[i + 2])),
               static_cast<float>(static_cast<int>(r[i + 3])), c, c, nb, nb);
+        pv[0] = ex2_approx(y[0]);
+        pv[1] = ex2_approx(y[1]);
+        if ((i & 4) == 0) {
+            pv[2] = ex2_approx(y[2]);
+            pv[3] = ex2_approx(y[3]);
+        } else {
+            exp2_poly2(y[2], y[3], pv[2], pv[3]);
+        }
+        if (MASK) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            pv[e] = ex2_approx(y[e]);
-            if (MASK && col0 + i + e >= n_valid) pv[e] = 0.f;
+            for (int e = 0; e < 4; ++e)
+                if (col0 + i + e >= n_valid) pv[e] = 0.f;
         }
         fadd2(acc[0], acc[1], acc[0], acc[1], pv[0], pv[1]);
         fadd2(acc[2], acc[3], acc[2], acc[3], pv[2], pv[3]);
@@ -254,23 +290,27 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         if (lane == 0) {
             const uint32_t idesc_qk = idesc_i8_s32(128, C::BN);
             const uint32_t idesc_pv = idesc_e4m3_f32_bmn(128, D);
-            const uint32_t q_addr = smem_u32(sQ);
-            const uint32_t p_addr = smem_u32(sP);
+            // Descriptors are built once; within a tile the start address field
+            // (address / 16 in the low bits, no carry for shared addresses) is
+            // advanced by plain additions.
+            const uint64_t dq = smem_desc_kmajor(smem_u32(sQ), D);
+            const uint64_t dk = smem_desc_kmajor(smem_u32(sK), D);
+            const uint64_t dv = smem_desc_mnmajor(smem_u32(sV), D);
+            const uint64_t dp = smem_desc_kmajor(smem_u32(sP), C::BN);
             auto issue_qk = [&](int t, int s) {
-                const uint32_t kb = smem_u32(sK + s * C::K_BYTES);
+                const uint64_t a = dq + (uint64_t)((t * C::Q_BYTES) >> 4);
+                const uint64_t b = dk + (uint64_t)((s * C::K_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 32; ++kk)
-                    mma_i8_ss(tmem + t * 128, smem_desc_kmajor(q_addr + t * C::Q_BYTES + kk * 32, D),
-                              smem_desc_kmajor(kb + kk * 32, D), idesc_qk, kk > 0 ? 1u : 0u);
+                    mma_i8_ss(tmem + t * 128, a + 2 * kk, b + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
                 tc_commit(&ctl->s_full[t]);
             };
             auto issue_pv = [&](int t, int s, int j) {
-                const uint32_t vb = smem_u32(sV + s * C::V_BYTES);
-                const uint32_t pb = p_addr + (2 * t + (j & 1)) * C::P_BYTES;
+                const uint64_t a = dp + (uint64_t)((((2 * t + (j & 1)) * C::P_BYTES)) >> 4);
+                const uint64_t b = dv + (uint64_t)((s * C::V_BYTES) >> 4);
 #pragma unroll
                 for (int kk = 0; kk < C::BN / 32; ++kk)
-                    mma_f8_ss(tmem + C::T_O + t * D, smem_desc_kmajor(pb + kk * 32, C::BN),
-                              smem_desc_mnmajor(vb + kk * 32 * D, D), idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                    mma_f8_ss(tmem + C::T_O + t * D, a + 2 * kk, b + 2 * kk * D, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
                 tc_commit(&ctl->o_done[t]);
                 if (j == nkv - 1) tc_commit(&ctl->o_final[t]);
             };
