@@ -287,66 +287,67 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         }
     } else if (warp == 9) {
         // ----------------------------------------------------------- MMA issue
-        if (lane == 0) {
-            const uint32_t idesc_qk = idesc_i8_s32(128, C::BN);
-            const uint32_t idesc_pv = idesc_e4m3_f32_bmn(128, D);
-            // Descriptors are built once; within a tile the start address field
-            // (address / 16 in the low bits, no carry for shared addresses) is
-            // advanced by plain additions.
-            const uint64_t dq = smem_desc_kmajor(smem_u32(sQ), D);
-            const uint64_t dk = smem_desc_kmajor(smem_u32(sK), D);
-            const uint64_t dv = smem_desc_mnmajor(smem_u32(sV), D);
-            const uint64_t dp = smem_desc_kmajor(smem_u32(sP), C::BN);
-            auto issue_qk = [&](int t, int s) {
-                const uint64_t a = dq + (uint64_t)((t * C::Q_BYTES) >> 4);
-                const uint64_t b = dk + (uint64_t)((s * C::K_BYTES) >> 4);
+        // The whole warp runs this loop (waits are warp-uniform); the elected
+        // lane issues the MMAs and commits.
+        const bool me = elect_one();
+        const uint32_t idesc_qk = idesc_i8_s32(128, C::BN);
+        const uint32_t idesc_pv = idesc_e4m3_f32_bmn(128, D);
+        // Descriptors are built once; within a tile the start address field
+        // (address / 16 in the low bits, no carry for shared addresses) is
+        // advanced by plain additions.
+        const uint64_t dq = smem_desc_kmajor(smem_u32(sQ), D);
+        const uint64_t dk = smem_desc_kmajor(smem_u32(sK), D);
+        const uint64_t dv = smem_desc_mnmajor(smem_u32(sV), D);
+        const uint64_t dp = smem_desc_kmajor(smem_u32(sP), C::BN);
+        auto issue_qk = [&](int t, int s) {
+            const uint64_t a = dq + (uint64_t)((t * C::Q_BYTES) >> 4);
+            const uint64_t b = dk + (uint64_t)((s * C::K_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 32; ++kk)
-                    mma_i8_ss(tmem + t * 128, a + 2 * kk, b + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
-                tc_commit(&ctl->s_full[t]);
-            };
-            auto issue_pv = [&](int t, int s, int j) {
-                const uint64_t a = dp + (uint64_t)((((2 * t + (j & 1)) * C::P_BYTES)) >> 4);
-                const uint64_t b = dv + (uint64_t)((s * C::V_BYTES) >> 4);
+            for (int kk = 0; kk < D / 32; ++kk)
+                mma_i8_ss_if(me, tmem + t * 128, a + 2 * kk, b + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
+            tc_commit_if(me, &ctl->s_full[t]);
+        };
+        auto issue_pv = [&](int t, int s, int j) {
+            const uint64_t a = dp + (uint64_t)((((2 * t + (j & 1)) * C::P_BYTES)) >> 4);
+            const uint64_t b = dv + (uint64_t)((s * C::V_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < C::BN / 32; ++kk)
-                    mma_f8_ss(tmem + C::T_O + t * D, a + 2 * kk, b + 2 * kk * D, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                tc_commit(&ctl->o_done[t]);
-                if (j == nkv - 1) tc_commit(&ctl->o_final[t]);
-            };
-            bool ok = wait_one(&ctl->q_full, 0, p.err, &ctl->abort, false, 4) &&
-                      wait_one(&ctl->kv_full[0], 0, p.err, &ctl->abort, false, 5);
-            if (ok) {
-                tc_fence_after();
-                issue_qk(0, 0);
-                issue_qk(1, 0);
-            }
-            for (int j = 0; ok && j < nkv; ++j) {
-                const int s = j % C::STAGES;
-                if (j + 1 < nkv) {
-                    const int s1 = (j + 1) % C::STAGES;
-                    if (!(ok = wait_one(&ctl->kv_full[s1], ((j + 1) / C::STAGES) & 1, p.err, &ctl->abort, false, 6)))
-                        break;
-                    for (int t = 0; ok && t < 2; ++t) {
-                        if (!(ok = wait_one(&ctl->s_free[t], j & 1, p.err, &ctl->abort, false, 7))) break;
-                        tc_fence_after();
-                        issue_qk(t, s1);  // the tile's softmax holds S(j) in registers already
-                    }
-                } else {
-                    for (int t = 0; ok && t < 2; ++t)
-                        ok = wait_one(&ctl->s_free[t], j & 1, p.err, &ctl->abort, false, 7);
-                }
-                for (int t = 0; ok && t < 2; ++t) {
-                    if (!(ok = wait_one(&ctl->p_ready[t][j & 1], (j >> 1) & 1, p.err, &ctl->abort, false, 8))) break;
-                    tc_fence_after();
-                    if (!EXPORT_S) issue_pv(t, s, j);
-                }
-                if (ok) tc_commit(&ctl->kv_empty[s]);
-            }
-            // all MMAs issued here finish before tensor memory is released
-            tc_commit(&ctl->drain);
-            wait_one(&ctl->drain, 0, p.err, &ctl->abort, true, 9);
+            for (int kk = 0; kk < C::BN / 32; ++kk)
+                mma_f8_ss_if(me, tmem + C::T_O + t * D, a + 2 * kk, b + 2 * kk * D, idesc_pv,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+            tc_commit_if(me, &ctl->o_done[t]);
+            if (j == nkv - 1) tc_commit_if(me, &ctl->o_final[t]);
+        };
+        bool ok = wait_warp(&ctl->q_full, 0, p.err, &ctl->abort, 4) &&
+                  wait_warp(&ctl->kv_full[0], 0, p.err, &ctl->abort, 5);
+        if (ok) {
+            tc_fence_after();
+            issue_qk(0, 0);
+            issue_qk(1, 0);
         }
+        for (int j = 0; ok && j < nkv; ++j) {
+            const int s = j % C::STAGES;
+            if (j + 1 < nkv) {
+                const int s1 = (j + 1) % C::STAGES;
+                if (!(ok = wait_warp(&ctl->kv_full[s1], ((j + 1) / C::STAGES) & 1, p.err, &ctl->abort, 6))) break;
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (!(ok = wait_warp(&ctl->s_free[t], j & 1, p.err, &ctl->abort, 7))) break;
+                    tc_fence_after();
+                    issue_qk(t, s1);  // the tile's softmax holds S(j) in registers already
+                }
+            } else {
+                for (int t = 0; ok && t < 2; ++t) ok = wait_warp(&ctl->s_free[t], j & 1, p.err, &ctl->abort, 7);
+            }
+            for (int t = 0; ok && t < 2; ++t) {
+                if (!(ok = wait_warp(&ctl->p_ready[t][j & 1], (j >> 1) & 1, p.err, &ctl->abort, 8))) break;
+                tc_fence_after();
+                if (!EXPORT_S) issue_pv(t, s, j);
+            }
+            if (ok) tc_commit_if(me, &ctl->kv_empty[s]);
+        }
+        // all MMAs issued here finish before tensor memory is released
+        tc_commit_if(me, &ctl->drain);
+        if (me) wait_one(&ctl->drain, 0, p.err, &ctl->abort, true, 9);
+        __syncwarp();
     } else if (warp < 8) {
         // ------------------------------------------------------------ softmax
         regs_increase<C::SOFTMAX_REGS>();
