@@ -444,14 +444,38 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     if (!(ok = wait_warp(&ctl->o_done[t], (j - 1) & 1, p.err, &ctl->abort, 12))) break;
                     tc_fence_after();
                     const float a = need ? alpha : 1.f;
-#pragma unroll 1
-                    for (int cc = 0; cc < D / 32; ++cc) {
-                        uint32_t o[32];
-                        tmem_ld_32x32b_x32(tO + cc * 32, o);
-                        tmem_wait_ld_x32(o);
+                    // the S registers are free again: load all of O's row at once
+                    tmem_ld_32x32b_x32(tO + 0, ra);
+                    tmem_ld_32x32b_x32(tO + 32, rb);
+                    if (D == 128) {
+                        tmem_ld_32x32b_x32(tO + 64, rc);
+                        tmem_ld_32x32b_x32(tO + 96, rd);
+                    }
+                    tmem_wait_ld_x32(ra);
+                    tmem_wait_ld_x32(rb);
+                    if (D == 128) {
+                        tmem_wait_ld_x32(rc);
+                        tmem_wait_ld_x32(rd);
+                    }
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * a);
-                        tmem_st_32x32b_x32(tO + cc * 32, o);
+                    for (int i = 0; i < 32; i += 2) {
+                        float x0, x1;
+                        fmul2(x0, x1, __uint_as_float(ra[i]), __uint_as_float(ra[i + 1]), a, a);
+                        ra[i] = __float_as_uint(x0), ra[i + 1] = __float_as_uint(x1);
+                        fmul2(x0, x1, __uint_as_float(rb[i]), __uint_as_float(rb[i + 1]), a, a);
+                        rb[i] = __float_as_uint(x0), rb[i + 1] = __float_as_uint(x1);
+                        if (D == 128) {
+                            fmul2(x0, x1, __uint_as_float(rc[i]), __uint_as_float(rc[i + 1]), a, a);
+                            rc[i] = __float_as_uint(x0), rc[i + 1] = __float_as_uint(x1);
+                            fmul2(x0, x1, __uint_as_float(rd[i]), __uint_as_float(rd[i + 1]), a, a);
+                            rd[i] = __float_as_uint(x0), rd[i + 1] = __float_as_uint(x1);
+                        }
+                    }
+                    tmem_st_32x32b_x32(tO + 0, ra);
+                    tmem_st_32x32b_x32(tO + 32, rb);
+                    if (D == 128) {
+                        tmem_st_32x32b_x32(tO + 64, rc);
+                        tmem_st_32x32b_x32(tO + 96, rd);
                     }
                     tmem_wait_st();
                 }
