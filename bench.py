@@ -148,39 +148,28 @@ def cpu_oracle_sample(w, seconds=12.0, seed=0):
 # --------------------------------------------------------------------------- GPU arm
 def run_gpu(args):
     import torch
-    import torch.distributed as dist
 
     import quantized_attention_qk_b200 as sage
     from quantized_attention_qk_b200 import build as sage_build
     from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv
+    from quantized_attention_qk_b200.replicas import Replicas, env_int, whole_job_tops
 
-    world = _env_int("WORLD_SIZE", 1)
-    rank = _env_int("RANK", 0)
-    local = _env_int("LOCAL_RANK", 0)
+    world = env_int("WORLD_SIZE", 1)
     if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
     if not torch.cuda.is_available():
         raise SystemExit("no CUDA device")
+    local = env_int("LOCAL_RANK", 0)
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    reps = Replicas(device=dev)
+    rank = reps.rank
     sage_build.build()
     sage.lib()
     peaks, peak_kind = _peaks()
     peak_8bit = 2.0 * float(peaks["bf16_tflops"])
-
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    barrier = reps.barrier
+    max_over_ranks = reps.max
 
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
 
@@ -243,7 +232,7 @@ def run_gpu(args):
     wp = WORKLOADS[args.workload]
     r = measure(wp, args.steps, args.warmup)
     ms = r["total_ms"] / args.steps
-    value = world * wp.ops * args.steps / (r["total_ms"] * 1e-3) / 1e12
+    value = whole_job_tops(world, wp.ops, args.steps, r["total_ms"])
     attn_tops = wp.ops / (r["attn_ms"] * 1e-3) / 1e12
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
@@ -267,7 +256,7 @@ def run_gpu(args):
         r2 = measure(ws_, max(3, args.steps // 2), args.warmup)
         k2 = max(3, args.steps // 2)
         line["secondary"] = {
-            "workload": _workload_desc(ws_), "value": round(world * ws_.ops * k2 / (r2["total_ms"] * 1e-3) / 1e12, 2),
+            "workload": _workload_desc(ws_), "value": round(whole_job_tops(world, ws_.ops, k2, r2["total_ms"]), 2),
             "unit": "TOPS", "ms_per_step": round(r2["total_ms"] / k2, 4), "steps": k2,
             "attn_tops": round(ws_.ops / (r2["attn_ms"] * 1e-3) / 1e12, 2), "attn_ms": round(r2["attn_ms"], 4),
             "attn_frac": round(ws_.ops / (r2["attn_ms"] * 1e-3) / 1e12 / peak_8bit, 4),
@@ -280,8 +269,7 @@ def run_gpu(args):
                                           f"included), {secs:.1f} s, quant-emulation mode"}
     if rank == 0:
         print(json.dumps(line, ensure_ascii=False), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    reps.close()
 
 
 # --------------------------------------------------------------------------- reference arm (the CPU oracle)

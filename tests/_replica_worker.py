@@ -1,0 +1,40 @@
+"""One rank of a CPU (gloo) replica group, started by test_replicas.py with the
+environment torchrun would give it.  Usage: _replica_worker.py MODE OUT_JSON"""
+import json
+import os
+import sys
+
+sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+
+from quantized_attention_qk_b200.replicas import Replicas, env_int, whole_job_tops  # noqa: E402
+
+
+def main():
+    mode, out = sys.argv[1], sys.argv[2]
+    rank = env_int("RANK", 0)
+    if mode == "never" and rank == 1:
+        sys.exit(0)  # this rank never joins the group
+    result = {"rank": rank}
+    try:
+        reps = Replicas(backend="gloo", timeout_s=float(os.environ.get("TEST_PG_TIMEOUT", "30")))
+        result["world"] = reps.world
+        if mode == "max":
+            # per-rank "times": rank r took 3 (r + 1) ms for 4 steps of 1e9 operations
+            t = reps.max(3.0 * (rank + 1))
+            reps.barrier()
+            result["max"] = t
+            result["tops"] = whole_job_tops(reps.world, 1e9, 4, t)
+        elif mode == "die":
+            if rank == 1:
+                os._exit(3)  # leaves between steps, before the next collective
+            reps.barrier()
+            result["max"] = reps.max(1.0)
+        reps.close()
+    except Exception as e:  # the error a surviving rank sees
+        result["error"] = type(e).__name__
+    with open(out, "w") as f:
+        json.dump(result, f)
+
+
+if __name__ == "__main__":
+    main()
