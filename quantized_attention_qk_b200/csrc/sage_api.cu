@@ -206,9 +206,9 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4], const
     c.q_scale = q_scale;
     c.k_i8 = k_i8;
     c.k_scale = k_scale;
-    cudaError_t e = launch_stats(s, &ks, nullptr, ws, k_mean, nullptr, st);
+    cudaError_t e = launch_stats(s, &ks, nullptr, ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, &ks, nullptr, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if ((e = launch_quant(s, &qs, &ks, nullptr, ws, k_mean, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
     return SAGE_OK;
 }
 
@@ -228,9 +228,9 @@ sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B,
     Codes c{};
     c.v_e4m3 = v_e4m3;
     c.v_scale = v_scale;
-    cudaError_t e = launch_stats(s, nullptr, &vs, ws, nullptr, v_scale, st);
+    cudaError_t e = launch_stats(s, nullptr, &vs, ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, nullptr, nullptr, &vs, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if ((e = launch_quant(s, nullptr, nullptr, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
     return SAGE_OK;
 }
 
@@ -279,9 +279,9 @@ sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4], const v
     const Codes c = carve_codes(scr.ptr, s);
     const StatsWs ws = carve_stats_ws(static_cast<char *>(scr.ptr) + cb, s);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_stats(s, &ks, &vs, ws, nullptr, c.v_scale, st);
+    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, &ks, &vs, ws, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if ((e = launch_quant(s, &qs, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_attention(s, c, dst(out, o_stride), sm_scale, st)) != cudaSuccess)

@@ -553,17 +553,6 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-unsigned *device_error_ptr() {
-    static unsigned *ptrs[64] = {nullptr};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!ptrs[dev]) {
-        void *a = nullptr;
-        if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
-        ptrs[dev] = static_cast<unsigned *>(a);
-    }
-    return ptrs[dev];
-}
 
 template <int D, bool EXPORT_S>
 cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
@@ -595,6 +584,48 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
 }
 
 }  // namespace
+
+unsigned *device_error_ptr() {
+    static unsigned *ptrs[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!ptrs[dev]) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
+        ptrs[dev] = static_cast<unsigned *>(a);
+    }
+    return ptrs[dev];
+}
+
+cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorSymbolNotFound;
+    // Dimensions after the channels: N and H in order of stride, then B.  A
+    // dimension of extent 1 is never stepped, so it gets the packed stride.
+    uint64_t st_n = (uint64_t)src.sn * 2, st_h = (uint64_t)src.sh * 2, st_b = (uint64_t)src.sb * 2;
+    bool swap;
+    if (s.H == 1) {
+        swap = false;
+        st_h = st_n * (uint64_t)s.N;
+    } else if (s.N == 1) {
+        swap = true;
+        st_n = st_h * (uint64_t)s.H;
+    } else {
+        swap = st_h < st_n;
+    }
+    const uint64_t e1 = swap ? s.H : s.N, e2 = swap ? s.N : s.H;
+    const uint64_t s1 = swap ? st_h : st_n, s2 = swap ? st_n : st_h;
+    if (s.B == 1) st_b = s2 * e2;
+    const cuuint64_t dims[4] = {(cuuint64_t)s.d, e1, e2, (cuuint64_t)s.B};
+    const cuuint64_t strides[3] = {s1, s2, st_b};
+    const cuuint32_t box[4] = {64, swap ? 1u : rows, swap ? rows : 1u, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t *>(src.p), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    *hn_swapped = swap ? 1 : 0;
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st) {
     AttnParams p{};

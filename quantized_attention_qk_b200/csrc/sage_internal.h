@@ -4,6 +4,7 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 namespace sage {
@@ -67,11 +68,18 @@ StatsWs carve_stats_ws(void *base, const Shape &s);
 size_t codes_bytes(const Shape &s);
 Codes carve_codes(void *base, const Shape &s);
 
-// Quantize pass launchers (sage_quant.cu).  `user_k_mean` may be null.
-cudaError_t launch_stats(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, float *user_k_mean,
-                         float *v_scale, cudaStream_t st);
+// Quantize pass launchers (sage_quant.cu): per-chunk partial statistics of K
+// and V, then the codes (the statistics are finished inside the second kernel).
+// `user_k_mean` may be null; the V scales go to c.v_scale.
+cudaError_t launch_stats(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, cudaStream_t st);
 cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                         const Codes &c, cudaStream_t st);
+                         float *user_k_mean, const Codes &c, cudaStream_t st);
+// 4-D tiled TMA map of a bf16 [B,H,N,d] view: box = 64 channels x `rows` tokens
+// of one (b,h).  The N and H dimensions are handed to the hardware in stride
+// order; *hn_swapped tells the kernel which coordinate comes second.
+cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped);
+// Device error word (bounded waits that gave up) of the current device.
+unsigned *device_error_ptr();
 
 // Attention launchers (sage_attn.cu).
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);
