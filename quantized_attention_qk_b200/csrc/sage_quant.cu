@@ -236,7 +236,10 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
     }
 }
 
-constexpr int kQThreads = 512;
+// Threads of a quantize CTA: 512 (one CTA per SM) for d = 128, 256 (two CTAs
+// per SM, so two items are in flight per SM) for d = 64.
+template <int D>
+__host__ __device__ constexpr int quant_threads() { return D == 128 ? 512 : 256; }
 
 // Persistent CTAs over the (b,h, 128-token block) items, a contiguous range
 // each (so consecutive items share a (b,h) and its statistics), two buffers:
@@ -252,11 +255,12 @@ struct QuantArgs {
 };
 
 template <int D, bool DO_Q, bool DO_K, bool DO_V>
-__global__ void __launch_bounds__(kQThreads, 1) k_quant(const __grid_constant__ CUtensorMap tq,
+__global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) k_quant(const __grid_constant__ CUtensorMap tq,
                                                         const __grid_constant__ CUtensorMap tk,
                                                         const __grid_constant__ CUtensorMap tv, const QuantArgs a) {
+    constexpr int NTH = quant_threads<D>();
     constexpr int VPR = D / 8;
-    constexpr int RPI = kQThreads / VPR;
+    constexpr int RPI = NTH / VPR;
     constexpr int NI = kQBlock / RPI;  // vectors per thread in one 128-token block
     constexpr int TILE = kQBlock * D;
     constexpr int NT = (DO_Q ? 1 : 0) + (DO_K ? 1 : 0) + (DO_V ? 1 : 0);
@@ -265,7 +269,7 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant(const __grid_constant__ 
     uint16_t *bufs = reinterpret_cast<uint16_t *>(smem_raw);  // [2][NT][TILE]
     __shared__ uint64_t bar[2];
     __shared__ float mu[D], vinv[D], vmax[D];
-    __shared__ float red[3 * (kQThreads / 32)];
+    __shared__ float red[3 * (NTH / 32)];
     __shared__ AbortState abort_st;
     __shared__ int bad;
     const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock;
@@ -307,7 +311,7 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant(const __grid_constant__ 
         if ((DO_K || DO_V) && bh != cur_bh) {
             // this (b,h)'s statistics from the chunk partials, in chunk order:
             // mean = sum / N (IEEE divide), V factor 448 / amax
-            for (int c = threadIdx.x; c < D; c += kQThreads) {
+            for (int c = threadIdx.x; c < D; c += NTH) {
                 float sum = 0.f, mx = 0.f;
 #pragma unroll 8
                 for (int ch = 0; ch < a.nch; ++ch) {
@@ -329,7 +333,7 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant(const __grid_constant__ 
         }
         __syncthreads();  // the rows and the statistics are ready
         if (blk == 0 && (DO_K || DO_V)) {
-            for (int c = threadIdx.x; c < D; c += kQThreads) {
+            for (int c = threadIdx.x; c < D; c += NTH) {
                 if (DO_K) {
                     a.ws_k_mean[bh * D + c] = mu[c];
                     if (a.user_k_mean) a.user_k_mean[bh * D + c] = mu[c];
@@ -378,7 +382,7 @@ __global__ void __launch_bounds__(kQThreads, 1) k_quant(const __grid_constant__ 
                     if (row < kKBlock) ka0 = fmaxf(ka0, am); else ka1 = fmaxf(ka1, am);
                 }
             }
-            block_max3_n<kQThreads>(qa, ka0, ka1, red);
+            block_max3_n<NTH>(qa, ka0, ka1, red);
         }
 
         if (DO_Q && !bad) {
@@ -496,10 +500,10 @@ cudaError_t launch_quant_k(const Shape &s, const CUtensorMap &tq, const CUtensor
         attr_set = true;
     }
     const int items = s.n_qblocks() * s.BH();
-    const int ctas = resident_ctas(kern, kQThreads, smem);
+    const int ctas = resident_ctas(kern, quant_threads<D>(), smem);
     if (ctas <= 0) return cudaErrorInvalidConfiguration;
     a.per = (items + ctas - 1) / ctas;
-    kern<<<(items + a.per - 1) / a.per, kQThreads, smem, st>>>(tq, tk, tv, a);
+    kern<<<(items + a.per - 1) / a.per, quant_threads<D>(), smem, st>>>(tq, tk, tv, a);
     return cudaGetLastError();
 }
 
