@@ -52,6 +52,25 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def _attn_traffic(workload):
+    """DRAM bytes per launch of the attention kernel, as counted by ncu on this
+    workload (profiles/k_attn_traffic.txt), or None when there is no count or
+    the kernel source changed since it was taken."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        with open(os.path.join(here, "profiles", "k_attn_traffic.txt")) as f:
+            rec = json.load(f)
+        with open(os.path.join(here, "quantized_attention_qk_b200", "csrc", "sage_attn.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    w = rec.get("workloads", {}).get(workload)
+    if rec.get("source_sha256") != sha or not w:
+        return None
+    return int(w["dram_bytes_read"]) + int(w["dram_bytes_write"])
+
+
 def _workload_desc(w):
     return f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.layout} qkv"
 
@@ -243,7 +262,7 @@ def run_gpu(args):
                    "l2": "flushed before every timed step (256 MB write, outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "k_attn (fused attention)", "achieved": round(attn_tops, 2),
                      "peak": round(peak_8bit, 1), "unit": "TFLOP/s", "frac": round(attn_tops / peak_8bit, 4),
-                     "traffic": None, "peak_source": f"{peak_kind}: {PEAK_NOTE}",
+                     "traffic": _attn_traffic(wp.name), "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
