@@ -213,6 +213,10 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
+// 8-byte shared-memory store.
+__device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
+    asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
+}
 __device__ __forceinline__ void tmem_wait_st() {
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -381,6 +385,31 @@ __device__ __forceinline__ void ffma2(float &d0, float &d1, float a0, float a1, 
         "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
         : "=f"(d0), "=f"(d1)
         : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+
+// bf16 pair packed in a 32-bit word -> two floats (element 2i in the low half).
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
+    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x);
+    f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
+    f[4] = bf_lo(u.z); f[5] = bf_hi(u.z);
+    f[6] = bf_lo(u.w); f[7] = bf_hi(u.w);
+}
+
+// Eight int8 codes rne(x * inv), saturated to [-128, 127], packed lowest byte
+// first into two words; the products come from packed fp32 multiplies (each an
+// IEEE-rounded product).  |x| <= amax makes |x * fp32(127/amax)| round to at
+// most 127, so the codes stay in [-127, 127] as the symmetric scheme requires.
+__device__ __forceinline__ uint2 i8x8(const float (&x)[8], float inv) {
+    float y[8];
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) fmul2(y[e], y[e + 1], x[e], x[e + 1], inv, inv);
+    uint32_t c[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(c[e]) : "f"(y[e]));
+    return make_uint2(__byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410),
+                      __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

@@ -27,17 +27,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// bf16 pair packed in a 32-bit word -> two floats (element 2i in the low half).
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8]) {
-    f[0] = bf_lo(u.x); f[1] = bf_hi(u.x);
-    f[2] = bf_lo(u.y); f[3] = bf_hi(u.y);
-    f[4] = bf_lo(u.z); f[5] = bf_hi(u.z);
-    f[6] = bf_lo(u.w); f[7] = bf_hi(u.w);
-}
-
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -71,21 +60,6 @@ __device__ __forceinline__ void load_rows(uint16_t *tile, int rows, const CUtens
             else
                 tma_load_4d_hint(dst, map, bar, half * 64, n + r, h, b, policy);
         }
-}
-
-// Eight int8 codes rne(x * inv), saturated to [-128, 127], packed lowest byte
-// first into two words; the products come from packed fp32 multiplies (each an
-// IEEE-rounded product).  |x| <= amax makes |x * fp32(127/amax)| round to at
-// most 127, so the codes stay in [-127, 127] as the symmetric scheme requires.
-__device__ __forceinline__ uint2 i8x8(const float (&x)[8], float inv) {
-    float y[8];
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) fmul2(y[e], y[e + 1], x[e], x[e + 1], inv, inv);
-    uint32_t c[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) asm("cvt.rni.sat.s8.f32 %0, %1;" : "=r"(c[e]) : "f"(y[e]));
-    return make_uint2(__byte_perm(__byte_perm(c[0], c[1], 0x0040), __byte_perm(c[2], c[3], 0x0040), 0x5410),
-                      __byte_perm(__byte_perm(c[4], c[5], 0x0040), __byte_perm(c[6], c[7], 0x0040), 0x5410));
 }
 
 // Max over the block of three values at once (all threads get the results).
@@ -534,6 +508,7 @@ cudaError_t launch_quant_d(const Shape &s, const Src *q, const Src *k, const Src
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
     if (q && k && v) return launch_quant_k<D, true, true, true>(s, tq, tk, tv, a, st);
     if (q && k && !v) return launch_quant_k<D, true, true, false>(s, tq, tk, tv, a, st);
+    if (!q && k && v) return launch_quant_k<D, false, true, true>(s, tq, tk, tv, a, st);
     if (!q && !k && v) return launch_quant_k<D, false, false, true>(s, tq, tk, tv, a, st);
     return cudaErrorInvalidValue;
 }

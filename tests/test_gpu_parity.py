@@ -204,6 +204,23 @@ def test_fused_and_contiguous_layouts_give_identical_bits():
     assert torch.equal(out_f.view(torch.int16), out_c.view(torch.int16))
 
 
+@pytest.mark.parametrize("N,d,layout", [(4608, 128, "fused"), (1000, 128, "contiguous"), (200, 64, "contiguous"),
+                                         (777, 64, "fused"), (129, 128, "fused"), (1, 64, "contiguous")])
+def test_prologue_q_quantization_matches_the_quantize_pass(N, d, layout):
+    """The forward quantizes Q inside the attention kernel; its output must be
+    bit-identical to the explicit path (quantize pass codes -> attention)."""
+    w = tiny_custom(1, 3, N, d, seed=40 + N, layout=layout, bias_sigma=4.0, outlier_frac=0.01)
+    _, (qd, kd, vd), _ = _inputs(w)
+    fused = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
+    c = sage.sage_quant_qk(qd, kd)
+    v_e4m3, v_scale = sage.sage_quant_v(vd)
+    explicit = sage.sage_attn_quantized(c["q_i8"], c["q_scale"], c["k_i8"], c["k_scale"], v_e4m3, v_scale, N,
+                                        sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(fused.view(torch.int16), explicit.view(torch.int16))
+
+
 def test_strided_output_and_explicit_workspace():
     w = tiny_custom(2, 2, 333, 64, seed=32, bias_sigma=2.0)
     _, (qd, kd, vd), _ = _inputs(w)
