@@ -200,6 +200,36 @@ sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4],
                                sage_stream_t stream,
                                sage_event_t attn_begin, sage_event_t attn_end);
 
+/* Layouts of the one host buffer that holds q, k and v for sage_attn_fwd_host. */
+#define SAGE_LAYOUT_FUSED 0      /* [B,N,3,H,d]: per token, the q, k and v rows of every head */
+#define SAGE_LAYOUT_CONTIGUOUS 1 /* [3,B,H,N,d]: q, then k, then v, each [B,H,N,d] */
+
+/* Bytes of device scratch sage_attn_fwd_host needs (0 for a shape it rejects):
+ * the input and output on the device plus two chunk workspaces. */
+size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d);
+
+/*
+ * sage_attn_fwd_host -- sage_attn_fwd on HOST memory, the end-to-end call:
+ * `qkv_host` (bf16, `layout` as above) goes to the device, the forward runs,
+ * and the bf16 result lands in `out_host` ([B,H,N,d] contiguous).  The heads
+ * are processed in chunks on two internal streams so that host<->device
+ * copies overlap the kernels of the other chunk; each chunk's result is the
+ * whole call's result for its heads, bit for bit (every statistic is per
+ * head).  Host buffers should be page-locked (cudaHostAlloc / pinned) for the
+ * copies to be asynchronous; pageable buffers work but serialise.
+ *   scratch: device buffer of >= sage_attn_fwd_host_scratch_bytes(B,H,N,d)
+ *            bytes, 256-byte aligned, or NULL (allocated and freed on `stream`).
+ * Enqueued after the work already on `stream`; `stream` continues after the
+ * whole call (out_host is complete once `stream` reaches that point).
+ * Errors: SAGE_ERR_INVALID_ARG (null buffer, layout, shape, sm_scale),
+ * SAGE_ERR_UNSUPPORTED (d), SAGE_ERR_WORKSPACE (scratch too small),
+ * SAGE_ERR_CUDA.  The pages have no counterpart; this is the call a serving
+ * path with host-resident tensors makes.
+ */
+sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_host,
+                                 int B, int H, int N, int d, float sm_scale,
+                                 void *scratch, size_t scratch_bytes, sage_stream_t stream);
+
 /*
  * sage_attn_dense_ref_gpu -- plain dense attention on the CUDA cores in fp32
  * ([SDPA] section 三.1, [H3] section 一): no quantization, no tensor cores,

@@ -56,6 +56,8 @@ _SIGS = {
     "sage_attn_dense_ref_gpu": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32,
                                  ctypes.c_float, _P], _I32),
     "sage_debug_qk_tile": ([_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
+    "sage_attn_fwd_host_scratch_bytes": ([_I32, _I32, _I32, _I32], _SZ),
+    "sage_attn_fwd_host": ([_P, _I32, _P, _I32, _I32, _I32, _I32, ctypes.c_float, _P, _SZ, _P], _I32),
 }
 
 
@@ -232,20 +234,40 @@ def sage_debug_qk_tile(q_i8, k_i8, N: int, b: int, h: int, q_tile: int, kv_tile:
     return s
 
 
+LAYOUTS = {"fused": 0, "contiguous": 1}  # SAGE_LAYOUT_FUSED, SAGE_LAYOUT_CONTIGUOUS
+
+
+def sage_attn_fwd_host_scratch_bytes(B, H, N, d):
+    return lib().sage_attn_fwd_host_scratch_bytes(B, H, N, d)
+
+
 def sage_attn_fwd_host(qkv_host, B, H, N, d, layout="fused", sm_scale=None, device="cuda", out_host=None,
                        workspace=None, stream=None):
-    """End-to-end call on HOST memory: copy the (pinned) input to the device,
-    run sage_attn_fwd, copy the bf16 result back into ``out_host``.
+    """End-to-end call on HOST memory (the library's sage_attn_fwd_host): the
+    bf16 input goes to the device chunk by chunk, the forward runs, and the bf16
+    result lands in ``out_host``.
 
-    ``qkv_host`` is one pinned bf16 buffer: [B,N,3,H,d] for layout "fused",
-    [3,B,H,N,d] for "contiguous".  Returns ``out_host`` ([B,H,N,d], pinned)."""
-    dev_buf = qkv_host.to(device, non_blocking=True)
-    if layout == "fused":
-        q, k, v = (dev_buf[:, :, i].permute(0, 2, 1, 3) for i in range(3))
-    else:
-        q, k, v = dev_buf[0], dev_buf[1], dev_buf[2]
-    out = sage_attn_fwd(q, k, v, sm_scale=sm_scale, workspace=workspace, stream=stream)
+    ``qkv_host`` is one contiguous bf16 host buffer: [B,N,3,H,d] for layout
+    "fused", [3,B,H,N,d] for "contiguous" (pinned for asynchronous copies).
+    ``workspace``: optional device scratch of sage_attn_fwd_host_scratch_bytes
+    bytes.  Returns ``out_host`` ([B,H,N,d]); it is complete once ``stream``
+    (default: the current stream of ``device``) reaches the end of the call."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"layout must be one of {sorted(LAYOUTS)}")
+    want = (B, N, 3, H, d) if layout == "fused" else (3, B, H, N, d)
+    if qkv_host.device.type != "cpu" or qkv_host.dtype != torch.bfloat16 or not qkv_host.is_contiguous() or \
+            tuple(qkv_host.shape) != want:
+        raise ValueError(f"qkv_host must be a contiguous bf16 host tensor of shape {want}")
     if out_host is None:
         out_host = torch.empty(B, H, N, d, dtype=torch.bfloat16, pin_memory=True)
-    out_host.copy_(out, non_blocking=True)
+    if out_host.device.type != "cpu" or out_host.dtype != torch.bfloat16 or not out_host.is_contiguous() or \
+            tuple(out_host.shape) != (B, H, N, d):
+        raise ValueError("out_host must be a contiguous bf16 host tensor of shape [B,H,N,d]")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    dev = torch.device(device)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(dev):
+        _raise(lib().sage_attn_fwd_host(_ptr(qkv_host), LAYOUTS[layout], _ptr(out_host), B, H, N, d,
+                                        ctypes.c_float(sm_scale), _ptr(workspace), ws_bytes, _stream(stream, dev)))
     return out_host

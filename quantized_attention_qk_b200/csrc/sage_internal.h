@@ -12,7 +12,7 @@ namespace sage {
 constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
 constexpr int kKBlock = 64;        // K tokens per quantization block
 constexpr int kKvTile = 128;       // keys per attention KV tile (two K blocks)
-constexpr int kStatsCtas = 592;    // statistics pass: aim for 4 CTAs per SM on 148 SMs
+constexpr int kStatsRows = 256;    // statistics pass: tokens per chunk (a multiple of 64)
 constexpr unsigned kErrTimeoutBit = 1u;  // device error word: a bounded wait gave up
 
 // A bf16 [B,H,N,d] tensor given by base pointer and element strides (c stride 1).
@@ -32,13 +32,10 @@ struct Shape {
     int n_qblocks() const { return n_pad() / kQBlock; }
     int n_kblocks() const { return n_pad() / kKBlock; }
     // Statistics pass: each (b,h) is cut into n_chunks() token chunks of
-    // chunk_rows() rows (a multiple of 64), enough CTAs to fill the GPU.
-    int chunk_rows() const {
-        int want = (kStatsCtas + BH() - 1) / BH();
-        int rows = (N + want - 1) / want;
-        rows = (rows + 63) / 64 * 64;
-        return rows < 64 ? 64 : rows;
-    }
+    // chunk_rows() rows.  The size depends on nothing but itself, so the fp32
+    // sums (and hence the codes) of a head do not depend on which other heads
+    // share the call.
+    int chunk_rows() const { return kStatsRows; }
     int n_chunks() const { return (N + chunk_rows() - 1) / chunk_rows(); }
 };
 

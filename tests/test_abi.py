@@ -84,3 +84,21 @@ def test_binding_raises_without_fallback(L):
     with pytest.raises(sage.SageError) as e:
         sage._raise(2)
     assert e.value.status == 2
+
+
+def test_host_forward_rejects_bad_arguments_before_any_launch(L):
+    buf = ctypes.create_string_buffer(4096)
+    p = ctypes.cast(buf, ctypes.c_void_p)
+    f = L.sage_attn_fwd_host
+    f.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                  ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    assert f(None, 0, p, 1, 1, 8, 64, 0.125, None, 0, None) == 1          # null input
+    assert f(p, 2, p, 1, 1, 8, 64, 0.125, None, 0, None) == 1             # unknown layout
+    assert f(p, 0, p, 1, 1, 8, 96, 0.125, None, 0, None) == 2             # head dim
+    assert f(p, 1, p, 1, 0, 8, 64, 0.125, None, 0, None) == 1             # shape
+    assert f(p, 1, p, 1, 1, 8, 64, float("nan"), None, 0, None) == 1      # sm_scale
+    assert f(p, 1, p, 1, 1, 8, 64, 0.125, p, 16, None) == 3               # scratch too small
+    L.sage_attn_fwd_host_scratch_bytes.restype = ctypes.c_size_t
+    assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 128) > 3 * 24 * 4608 * 128 * 2 + 24 * 4608 * 128 * 2
+    assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 96) == 0

@@ -221,6 +221,27 @@ def test_prologue_q_quantization_matches_the_quantize_pass(N, d, layout):
     assert torch.equal(fused.view(torch.int16), explicit.view(torch.int16))
 
 
+@pytest.mark.parametrize("B,H,N,d,layout,pinned", [(1, 24, 1000, 128, "fused", True), (2, 5, 777, 64, "contiguous", True),
+                                                   (2, 3, 300, 128, "fused", False), (1, 1, 129, 64, "fused", True)])
+def test_host_memory_forward_matches_the_device_forward(B, H, N, d, layout, pinned):
+    """sage_attn_fwd_host (head chunks on two streams, host<->device copies
+    inside) gives the device forward's bits."""
+    w = tiny_custom(B, H, N, d, seed=70 + N, layout=layout, bias_sigma=4.0, outlier_frac=0.01)
+    _, (qd, kd, vd), bufs = _inputs(w)
+    want = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
+    host_in = (bufs[0] if layout == "fused" else torch.stack(bufs)).cpu()
+    if pinned:
+        host_in = host_in.pin_memory()
+    got = sage.sage_attn_fwd_host(host_in, B, H, N, d, layout=layout, sm_scale=w.sm_scale, device=DEV)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(got.view(torch.int16), want.cpu().view(torch.int16))
+    small = torch.empty(64, dtype=torch.uint8, device=DEV)
+    with pytest.raises(sage.SageError) as e:
+        sage.sage_attn_fwd_host(host_in, B, H, N, d, layout=layout, sm_scale=w.sm_scale, device=DEV, workspace=small)
+    assert e.value.status == 3
+
+
 def test_strided_output_and_explicit_workspace():
     w = tiny_custom(2, 2, 333, 64, seed=32, bias_sigma=2.0)
     _, (qd, kd, vd), _ = _inputs(w)
