@@ -1,7 +1,7 @@
 // sage_host.cu -- the forward on host memory.  The heads are cut into chunks
 // that flow through host->device copies, the quantize and attention kernels
-// and the device->host copy of their output on two internal streams, so the
-// copies of one chunk overlap the kernels of the other (copies in both
+// and the device->host copy of their output on a few internal streams, so the
+// copies of one chunk overlap the kernels of another (copies in both
 // directions use their own copy engines).  Every chunk computes exactly what
 // the whole call would for its heads: all statistics are per head.
 #include <cuda_runtime.h>
@@ -18,22 +18,32 @@ namespace {
 constexpr size_t kAlign = 1024;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Heads per chunk: about four chunks per batch row, at least one head.
-int chunk_heads(int H) { return (H + 3) / 4; }
+constexpr int kStreams = 3;  // internal streams (and chunk workspaces)
+
+// Heads per chunk: about 64 MiB of input per chunk, between 4 and 16 chunks
+// per call (small chunks make the strided copies of a fused layout slow; few
+// chunks leave the first copy and the last kernels unoverlapped).
+int chunk_heads(int B, int H, int N, int d) {
+    const double in_bytes = 6.0 * B * H * N * d;
+    int chunks = static_cast<int>(in_bytes / (64.0 * 1024 * 1024)) + 1;
+    chunks = chunks < 4 ? 4 : (chunks > 16 ? 16 : chunks);
+    const int per_row = (chunks + B - 1) / B;  // chunks of each batch row
+    return (H + per_row - 1) / per_row;
+}
 
 size_t chunk_ws_bytes(int hc, int N, int d) {
     const Shape cs{1, hc, N, d};
     return up(codes_bytes(cs)) + up(stats_ws_bytes(cs));
 }
 
-// Two non-blocking streams per device, created on first use and kept for the
-// life of the process.
+// kStreams non-blocking streams per device, created on first use and kept for
+// the life of the process.
 struct DeviceStreams {
-    cudaStream_t s[2] = {nullptr, nullptr};
+    cudaStream_t s[kStreams] = {};
     bool ready = false;
 };
 
-cudaError_t device_streams(cudaStream_t (&out)[2]) {
+cudaError_t device_streams(cudaStream_t (&out)[kStreams]) {
     static std::mutex mu;
     static DeviceStreams per_dev[64];
     int dev = 0;
@@ -43,19 +53,18 @@ cudaError_t device_streams(cudaStream_t (&out)[2]) {
     std::lock_guard<std::mutex> lock(mu);
     DeviceStreams &ds = per_dev[dev];
     if (!ds.ready) {
-        for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < kStreams; ++i)
             if ((e = cudaStreamCreateWithFlags(&ds.s[i], cudaStreamNonBlocking)) != cudaSuccess) return e;
         ds.ready = true;
     }
-    out[0] = ds.s[0];
-    out[1] = ds.s[1];
+    for (int i = 0; i < kStreams; ++i) out[i] = ds.s[i];
     return cudaSuccess;
 }
 
 // Events of one call, released when the call's work is enqueued (an event
 // may be destroyed while work waiting on it is still pending).
 struct Events {
-    cudaEvent_t ev[3] = {nullptr, nullptr, nullptr};
+    cudaEvent_t ev[1 + kStreams] = {};
     ~Events() {
         for (cudaEvent_t e : ev)
             if (e) cudaEventDestroy(e);
@@ -72,7 +81,7 @@ extern "C" {
 size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d) {
     if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
     const size_t elems = (size_t)B * H * N * d;
-    return up(3 * elems * 2) + up(elems * 2) + 2 * chunk_ws_bytes(chunk_heads(H), N, d);
+    return up(3 * elems * 2) + up(elems * 2) + kStreams * chunk_ws_bytes(chunk_heads(B, H, N, d), N, d);
 }
 
 sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_host, int B, int H, int N, int d,
@@ -111,7 +120,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
         set_last_error("%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
         return SAGE_ERR_CUDA;
     };
-    cudaStream_t st[2];
+    cudaStream_t st[kStreams];
     cudaError_t e = device_streams(st);
     if (e != cudaSuccess) return cuda_fail(e, "internal streams");
     bool owned = false;
@@ -124,25 +133,26 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
         if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
     // the internal streams start after everything already on the caller's stream
     if ((e = cudaEventRecord(ev.ev[0], user)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < kStreams; ++i)
         if ((e = cudaStreamWaitEvent(st[i], ev.ev[0], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
 
     const size_t elems = (size_t)B * H * N * d;
     char *base = static_cast<char *>(scratch);
     uint16_t *d_in = reinterpret_cast<uint16_t *>(base);
     uint16_t *d_out = reinterpret_cast<uint16_t *>(base + up(3 * elems * 2));
-    const int hc_max = chunk_heads(H);
-    char *ws[2] = {base + up(3 * elems * 2) + up(elems * 2),
-                   base + up(3 * elems * 2) + up(elems * 2) + chunk_ws_bytes(hc_max, N, d)};
+    const int hc_max = chunk_heads(B, H, N, d);
+    char *ws0 = base + up(3 * elems * 2) + up(elems * 2);
+    const size_t ws_step = chunk_ws_bytes(hc_max, N, d);
     const uint16_t *h_in = static_cast<const uint16_t *>(qkv_host);
     uint16_t *h_out = static_cast<uint16_t *>(out_host);
     const int64_t hd = (int64_t)H * d, nd = (int64_t)N * d;
 
-    int c = 0;  // chunk count: chunk c runs on stream c % 2 with workspace c % 2
+    int c = 0;  // chunk count: chunk c runs on stream c % kStreams with that stream's workspace
     for (int b = 0; b < B; ++b)
         for (int h0 = 0; h0 < H; h0 += hc_max, ++c) {
             const int hc = H - h0 < hc_max ? H - h0 : hc_max;
-            cudaStream_t s = st[c & 1];
+            cudaStream_t s = st[c % kStreams];
+            char *ws = ws0 + (c % kStreams) * ws_step;
             const Shape cs{1, hc, N, d};
             Src q, k, v;
             if (layout == SAGE_LAYOUT_FUSED) {
@@ -172,8 +182,8 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
             }
             const int64_t ooff = ((int64_t)b * H + h0) * nd;
             const Dst o{d_out + ooff, (int64_t)H * nd, nd, d};
-            const Codes codes = carve_codes(ws[c & 1], cs);
-            const StatsWs sw = carve_stats_ws(ws[c & 1] + up(codes_bytes(cs)), cs);
+            const Codes codes = carve_codes(ws, cs);
+            const StatsWs sw = carve_stats_ws(ws + up(codes_bytes(cs)), cs);
             if ((e = launch_stats(cs, &k, &v, sw, s)) != cudaSuccess) return cuda_fail(e, "statistics pass");
             if ((e = launch_quant(cs, &q, &k, &v, sw, nullptr, codes, s)) != cudaSuccess)
                 return cuda_fail(e, "quantize pass");
@@ -183,7 +193,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
                 return cuda_fail(e, "device-to-host copy");
         }
     // the caller's stream continues after both internal streams
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kStreams; ++i) {
         if ((e = cudaEventRecord(ev.ev[1 + i], st[i])) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
         if ((e = cudaStreamWaitEvent(user, ev.ev[1 + i], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
     }
