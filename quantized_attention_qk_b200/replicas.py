@@ -1,10 +1,16 @@
-"""Coordination of replicas when the forward runs on several GPUs of one node.
+"""Running the forward on several GPUs of one node.
 
 The attention of one (batch, head) pair needs nothing from any other, so the
-GPUs share no data: every rank runs its own replica of the workload on its own
-device and the ranks only agree on timing (a barrier on both sides of the timed
-region and the maximum of the per-rank times).  The job's throughput is then
-the work of all ranks divided by that maximum (weak scaling).
+GPUs share no data on the way in.  Two uses:
+
+* replicas (what bench.py measures): every rank runs its own copy of the
+  workload and the ranks only agree on timing (a barrier on both sides of the
+  timed region and the maximum of the per-rank times); the job's throughput is
+  the work of all ranks divided by that maximum (weak scaling);
+* head sharding (`sharded_forward`): one problem split by heads, rank r
+  computing heads `head_range(H, world, r)` of every batch row on its own
+  device, optionally followed by one all-gather of the bf16 outputs so that
+  every rank holds the whole result (strong scaling).
 
 One process per GPU, launched by torchrun (RANK, LOCAL_RANK, WORLD_SIZE,
 MASTER_ADDR, MASTER_PORT in the environment).  NCCL carries the two collectives
@@ -76,3 +82,45 @@ def whole_job_tops(world: int, ops_per_step: float, steps: int, max_total_ms: fl
     if max_total_ms <= 0:
         raise ValueError("the timed region must have a positive duration")
     return world * ops_per_step * steps / (max_total_ms * 1e-3) / 1e12
+
+
+def head_range(H: int, world: int, rank: int) -> tuple[int, int]:
+    """Heads [h0, h1) of `rank` when H heads are split over `world` ranks as
+    evenly as possible (the first H mod world ranks take one more)."""
+    base, extra = divmod(H, world)
+    h0 = rank * base + min(rank, extra)
+    return h0, h0 + base + (1 if rank < extra else 0)
+
+
+def sharded_forward(q, k, v, reps: Replicas, sm_scale=None, gather: bool = True, attn=None, out_dtype=None):
+    """Head-sharded forward of one problem over the ranks of `reps`.
+
+    Every rank holds q, k, v ([B,H,N,d] views, any strides) and computes its
+    heads `head_range(H, world, rank)` of every batch row through `attn`
+    (default: the library's sage_attn_fwd) on strided views of them, without
+    copies.  With `gather` the ranks then exchange their outputs (one
+    all-gather, outputs padded to the largest share) and each returns the
+    whole [B,H,N,d] result; without it each returns its own [B,h1-h0,N,d]
+    part.  A rank whose share is empty computes nothing.  `out_dtype` is the
+    dtype `attn` returns (default q's, as sage_attn_fwd does); an empty share
+    takes it, so that all ranks gather the same type."""
+    if attn is None:
+        from quantized_attention_qk_b200 import sage_attn_fwd as attn
+    B, H, N, d = q.shape
+    h0, h1 = head_range(H, reps.world, reps.rank)
+    if h1 > h0:
+        part = attn(q[:, h0:h1], k[:, h0:h1], v[:, h0:h1], sm_scale=sm_scale)
+    else:
+        part = torch.empty(B, 0, N, d, dtype=out_dtype or q.dtype, device=q.device)
+    if not gather or reps.world == 1:
+        return part
+    hmax = -(-H // reps.world)
+    buf = torch.zeros(B, hmax, N, d, dtype=part.dtype, device=part.device)
+    buf[:, : h1 - h0] = part
+    parts = [torch.empty_like(buf) for _ in range(reps.world)]
+    dist.all_gather(parts, buf)
+    out = torch.empty(B, H, N, d, dtype=part.dtype, device=part.device)
+    for r in range(reps.world):
+        a, b = head_range(H, reps.world, r)
+        out[:, a:b] = parts[r][:, : b - a]
+    return out

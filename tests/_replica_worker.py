@@ -6,7 +6,7 @@ import sys
 
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 
-from quantized_attention_qk_b200.replicas import Replicas, env_int, whole_job_tops  # noqa: E402
+from quantized_attention_qk_b200.replicas import Replicas, env_int, head_range, sharded_forward, whole_job_tops  # noqa: E402
 
 
 def main():
@@ -24,6 +24,25 @@ def main():
             reps.barrier()
             result["max"] = t
             result["tops"] = whole_job_tops(reps.world, 1e9, 4, t)
+        elif mode.startswith("shard"):
+            # one problem split by heads; the compute is the oracle's exact
+            # attention (the sharding and the gather are what is tested)
+            import torch
+            import oracle
+            H = int(mode[len("shard"):])
+            g = torch.Generator().manual_seed(5)
+            q, k, v = (torch.randn(2, H, 40, 16, generator=g).to(torch.bfloat16) for _ in range(3))
+
+            def attn(qs, ks, vs, sm_scale=None):
+                return torch.from_numpy(oracle.attn_exact(qs, ks, vs, sm_scale))
+
+            full = sharded_forward(q, k, v, reps, sm_scale=0.25, gather=True, attn=attn, out_dtype=torch.float64)
+            part = sharded_forward(q, k, v, reps, sm_scale=0.25, gather=False, attn=attn, out_dtype=torch.float64)
+            ref = attn(q, k, v, sm_scale=0.25)
+            h0, h1 = head_range(H, reps.world, rank)
+            result["gathered_equal"] = bool(torch.equal(full, ref))
+            result["part_equal"] = bool(torch.equal(part, ref[:, h0:h1]))
+            result["heads"] = [h0, h1]
         elif mode == "die":
             if rank == 1:
                 os._exit(3)  # leaves between steps, before the next collective

@@ -242,6 +242,23 @@ def test_host_memory_forward_matches_the_device_forward(B, H, N, d, layout, pinn
     assert e.value.status == 3
 
 
+@pytest.mark.parametrize("world", [2, 3])
+def test_head_shares_reproduce_the_whole_forward(world):
+    """Each rank's head share (as sharded_forward computes it, on strided
+    views) equals the whole forward's heads bit for bit: the shares of a
+    head-sharded run need no communication but the final gather."""
+    from types import SimpleNamespace
+    from quantized_attention_qk_b200.replicas import head_range, sharded_forward
+    w = tiny_custom(2, 5, 700, 128, seed=81, layout="fused", bias_sigma=4.0, outlier_frac=0.01)
+    _, (qd, kd, vd), _ = _inputs(w)
+    whole = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
+    for r in range(world):
+        part = sharded_forward(qd, kd, vd, SimpleNamespace(world=world, rank=r), sm_scale=w.sm_scale, gather=False)
+        h0, h1 = head_range(5, world, r)
+        torch.cuda.synchronize()
+        assert torch.equal(part.view(torch.int16), whole[:, h0:h1].view(torch.int16))
+
+
 def test_strided_output_and_explicit_workspace():
     w = tiny_custom(2, 2, 333, 64, seed=32, bias_sigma=2.0)
     _, (qd, kd, vd), _ = _inputs(w)

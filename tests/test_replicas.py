@@ -9,7 +9,7 @@ import sys
 
 import pytest
 
-from quantized_attention_qk_b200.replicas import Replicas, whole_job_tops
+from quantized_attention_qk_b200.replicas import Replicas, head_range, whole_job_tops
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
@@ -94,3 +94,22 @@ def test_reference_arm_does_nothing_on_other_ranks():
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert p.returncode == 0
     assert p.stdout.strip() == ""
+
+
+def test_head_ranges_cover_every_head_once():
+    for H in (1, 2, 5, 24, 40):
+        for W in (1, 2, 3, 8):
+            got = [head_range(H, W, r) for r in range(W)]
+            assert got[0][0] == 0 and got[-1][1] == H
+            assert all(a[1] == b[0] for a, b in zip(got, got[1:]))
+            sizes = [b - a for a, b in got]
+            assert max(sizes) - min(sizes) <= 1
+
+
+@pytest.mark.parametrize("world,H", [(2, 5), (3, 5), (2, 1)])
+def test_head_sharded_forward_gathers_the_whole_result(tmp_path, world, H):
+    codes, res = _run_ranks(f"shard{H}", tmp_path, world=world)
+    assert codes == [0] * world
+    for r in res:
+        assert "error" not in r, r
+        assert r["gathered_equal"] and r["part_equal"], r
