@@ -43,7 +43,7 @@ def build(force: bool = False) -> str:
 
 class _Flags(ctypes.Structure):
     _fields_ = [("int8_qk", ctypes.c_int), ("fp8_p", ctypes.c_int), ("fp8_v", ctypes.c_int),
-                ("round_bf16", ctypes.c_int), ("smooth_k", ctypes.c_int)]
+                ("round_bf16", ctypes.c_int), ("smooth_k", ctypes.c_int), ("k_residual", ctypes.c_int)]
 
 
 _lib = None
@@ -59,10 +59,12 @@ def lib():
         L.oracle_attn_quant.argtypes = [P, I64, P, I64, P, I64, I32, I32, ctypes.c_float,
                                         ctypes.POINTER(_Flags), P, I32, P, P]
         L.oracle_int8_gemm_nt.argtypes = [P, I64, P, I64, I32, I32, I32, P]
+        L.oracle_quantize_kres.argtypes = [P, I64, I32, I32, P, P, P]
         L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         L.oracle_e4m3_decode_array.argtypes = [P, I64, P]
         L.oracle_bf16_rne_array.argtypes = [P, I64, P]
-        for f in ("oracle_attn_exact", "oracle_quantize", "oracle_attn_quant", "oracle_int8_gemm_nt"):
+        for f in ("oracle_attn_exact", "oracle_quantize", "oracle_attn_quant", "oracle_int8_gemm_nt",
+                  "oracle_quantize_kres"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -144,13 +146,35 @@ def quantize(q, k, v, smooth_k=True):
     return res
 
 
+def quantize_kres(k):
+    """K-residual codes of every slab ("ComfyUI-sol-attn", 核心亮点 item 1).
+    Returns dict k_i8 [B,H,N,d] int8, k_scale [B,H,ceil(N/64)] f32,
+    k_bmean [B,H,ceil(N/64),d] bf16 bit patterns (uint16)."""
+    B, H, N, d = k.shape
+    nkb = -(-N // K_BLOCK)
+    res = dict(k_i8=np.zeros((B, H, N, d), np.int8), k_scale=np.zeros((B, H, nkb), np.float32),
+               k_bmean=np.zeros((B, H, nkb, d), np.uint16))
+    L = lib()
+    for b in range(B):
+        for h in range(H):
+            kp, ks = _slab(k, b, h)
+            slab = {kk: np.ascontiguousarray(vv[b, h]) for kk, vv in res.items()}
+            _check(L.oracle_quantize_kres(kp, ks, N, d, _ptr(slab["k_i8"]), _ptr(slab["k_scale"]),
+                                          _ptr(slab["k_bmean"])), "quantize_kres")
+            for kk in res:
+                res[kk][b, h] = slab[kk]
+    return res
+
+
 def attn_quant(q, k, v, sm_scale, rows=None, int8_qk=True, fp8_p=True, fp8_v=True,
-               round_bf16=True, smooth_k=True, heads=None):
+               round_bf16=True, smooth_k=True, heads=None, k_residual=False):
     """Quant-emulation attention.  Returns (out_f64 [B,H,R,d], out_bf16 bits [B,H,R,d] uint16).
-    ``heads`` optionally restricts the work to a list of (b, h) pairs (others stay zero)."""
+    ``heads`` optionally restricts the work to a list of (b, h) pairs (others stay zero).
+    ``k_residual``: K-residual quantization with the block-mean term kept
+    (oracle_quantize_kres) instead of the smoothing."""
     B, H, N, d = q.shape
     r = _rows_array(rows, N)
-    f = _Flags(int(int8_qk), int(fp8_p), int(fp8_v), int(round_bf16), int(smooth_k))
+    f = _Flags(int(int8_qk), int(fp8_p), int(fp8_v), int(round_bf16), int(smooth_k), int(k_residual))
     out = np.zeros((B, H, len(r), d), dtype=np.float64)
     outb = np.zeros((B, H, len(r), d), dtype=np.uint16)
     L = lib()

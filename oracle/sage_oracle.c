@@ -27,6 +27,10 @@
  * Two modes:
  *   oracle_attn_exact  -- the plain definition in fp64 (no smoothing, no
  *                         quantization).
+ *   (oracle_attn_quant with k_residual set follows "ComfyUI-sol-attn",
+ *   核心亮点 item 1 instead of the smoothing: only the residual of K inside
+ *   each 64-token block is quantized, and the block mean term stays at bf16
+ *   precision -- see oracle_quantize_kres.)
  *   oracle_attn_quant  -- the quantization scheme, step by step, in the order
  *                         smoothing -> block INT8 of Q and K -> integer Q K^T ->
  *                         dequant -> softmax with an integer-grid (log2) row max
@@ -304,6 +308,47 @@ int oracle_quantize(const uint16_t *q, int64_t q_rs,
     return 0;
 }
 
+/*
+ * K-residual quantization of K for one slab ("ComfyUI-sol-attn", 核心亮点
+ * item 1: quantize only the residual of K inside each block, keep the mean
+ * term at bf16 precision).  Readings where the page is silent: the blocks are
+ * the 64-token K blocks of reading C3; the block mean is the fp64 mean over
+ * the block's valid tokens, rounded to bf16 (RNE); the residual k - mean is
+ * formed in fp32 (exact: both are bf16 values) and coded as in reading C2 with
+ * the block's amax of the residual.
+ *   k_bmean[nkb][d] (bf16 bit patterns), k_i8[N][d], k_scale[nkb].
+ */
+int oracle_quantize_kres(const uint16_t *k, int64_t k_rs, int N, int d,
+                         int8_t *k_i8, float *k_scale, uint16_t *k_bmean)
+{
+    if (N <= 0 || d <= 0) return -1;
+    int nkb = (N + ORACLE_K_BLOCK - 1) / ORACLE_K_BLOCK;
+    for (int b = 0; b < nkb; ++b) {
+        int n0 = b * ORACLE_K_BLOCK, n1 = n0 + ORACLE_K_BLOCK;
+        if (n1 > N) n1 = N;
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int n = n0; n < n1; ++n) acc += oracle_bf16_to_double(k[(int64_t)n * k_rs + c]);
+            k_bmean[(size_t)b * d + c] = oracle_bf16_rne(acc / (double)(n1 - n0));
+        }
+        float amax = 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float r = bf16_to_float(k[(int64_t)n * k_rs + c]) - bf16_to_float(k_bmean[(size_t)b * d + c]);
+                float a = fabsf(r);
+                if (a > amax) amax = a;
+            }
+        float inv = amax > 0.0f ? 127.0f / amax : 0.0f;
+        k_scale[b] = amax > 0.0f ? amax / 127.0f : 0.0f;
+        for (int n = n0; n < n1; ++n)
+            for (int c = 0; c < d; ++c) {
+                float r = bf16_to_float(k[(int64_t)n * k_rs + c]) - bf16_to_float(k_bmean[(size_t)b * d + c]);
+                k_i8[(int64_t)n * d + c] = amax > 0.0f ? int8_code(r, inv) : 0;
+            }
+    }
+    return 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Quant-emulation attention                                                */
 /* ------------------------------------------------------------------------ */
@@ -315,6 +360,8 @@ typedef struct {
     int fp8_v;      /* 0: V kept exact (no e4m3, no scale)                      */
     int round_bf16; /* 0: out_bf16 still written, but from the unrounded value */
     int smooth_k;   /* 0: no mean subtraction before K quantization            */
+    int k_residual; /* 1: K-residual quantization (oracle_quantize_kres) instead
+                       of the smoothing; the scores then add q.mean_block     */
 } oracle_quant_flags;
 
 /*
@@ -329,7 +376,10 @@ typedef struct {
  *   O_rc   = sum_j P_rj * vcode_value[j,c]                 (fp64)
  *   out_rc = bf16_rne( O_rc * v_scale[c] / (448 l_r) )    (reading C8)
  * The dropped smoothing term q.mean is a per-row constant of the scores and
- * cancels in the softmax (reading C1).  Because m_r lies on the integer grid,
+ * cancels in the softmax (reading C1).  With k_residual the K codes are those
+ * of oracle_quantize_kres and x_rj gains e_rb = (q_r . mean_b) * sm_scale *
+ * log2 e for the key's block b (fp64 from the bf16 values): that term varies
+ * with the block, so it is kept, at the mean's bf16 precision.  Because m_r lies on the integer grid,
  * a tiled online evaluation that rescales by 2^(m_old - m_new) produces the
  * same P codes as this one-pass form wherever 448 p stays in e4m3's normal
  * range (reading C5); below it (448 p < 2^-6) the one-pass form is used.
@@ -355,11 +405,14 @@ int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
     double *x = (double *)malloc(sizeof(double) * (size_t)N);
     double *vval = (double *)malloc(sizeof(double) * nd);
     double *o = (double *)malloc(sizeof(double) * (size_t)d);
+    uint16_t *kbm = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)nkb * d);
+    double *e = (double *)malloc(sizeof(double) * (size_t)nkb);
     int rc = 0;
-    if (!qc || !kc || !vc || !qs || !ks || !km || !vs || !x || !vval || !o) { rc = -2; goto done; }
+    if (!qc || !kc || !vc || !qs || !ks || !km || !vs || !x || !vval || !o || !kbm || !e) { rc = -2; goto done; }
 
-    rc = oracle_quantize(q, q_rs, k, k_rs, v, v_rs, N, d, flags->smooth_k,
+    rc = oracle_quantize(q, q_rs, k, k_rs, v, v_rs, N, d, flags->k_residual ? 0 : flags->smooth_k,
                          qc, qs, kc, ks, km, vc, vs);
+    if (!rc && flags->k_residual) rc = oracle_quantize_kres(k, k_rs, N, d, kc, ks, kbm);
     if (rc) goto done;
 
     /* value of V used in the P.V product, already multiplied by its scale */
@@ -378,20 +431,31 @@ int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
         float sq = qs[r / ORACLE_Q_BLOCK];
         float cq = sq * s_l2; /* fp32 */
         double xmax = -INFINITY;
+        for (int b = 0; b < nkb; ++b) {
+            double acc = 0.0;
+            if (flags->k_residual)
+                for (int c = 0; c < d; ++c)
+                    acc += oracle_bf16_to_double(q[(int64_t)r * q_rs + c]) *
+                           oracle_bf16_to_double(kbm[(size_t)b * d + c]);
+            e[b] = acc * (double)sm_scale * 1.4426950408889634;
+        }
         for (int j = 0; j < N; ++j) {
             if (flags->int8_qk) {
                 int64_t S = 0;
                 for (int c = 0; c < d; ++c)
                     S += (int64_t)qc[(size_t)r * d + c] * (int64_t)kc[(size_t)j * d + c];
                 float cj = cq * ks[j / ORACLE_K_BLOCK]; /* fp32 */
-                x[j] = (double)S * (double)cj;
+                x[j] = (double)S * (double)cj + e[j / ORACLE_K_BLOCK];
             } else {
                 double acc = 0.0;
-                for (int c = 0; c < d; ++c)
-                    acc += oracle_bf16_to_double(q[(int64_t)r * q_rs + c]) *
-                           (oracle_bf16_to_double(k[(int64_t)j * k_rs + c]) -
-                            (flags->smooth_k ? (double)km[c] : 0.0));
-                x[j] = acc * (double)sm_scale * 1.4426950408889634;
+                for (int c = 0; c < d; ++c) {
+                    const double kj = oracle_bf16_to_double(k[(int64_t)j * k_rs + c]);
+                    const double sub = flags->k_residual
+                                           ? oracle_bf16_to_double(kbm[(size_t)(j / ORACLE_K_BLOCK) * d + c])
+                                           : (flags->smooth_k ? (double)km[c] : 0.0);
+                    acc += oracle_bf16_to_double(q[(int64_t)r * q_rs + c]) * (kj - sub);
+                }
+                x[j] = acc * (double)sm_scale * 1.4426950408889634 + e[j / ORACLE_K_BLOCK];
             }
             if (x[j] > xmax) xmax = x[j];
         }
@@ -413,7 +477,7 @@ int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
     }
 done:
     free(qc); free(kc); free(vc); free(qs); free(ks); free(km); free(vs);
-    free(x); free(vval); free(o);
+    free(x); free(vval); free(o); free(kbm); free(e);
     return rc;
 }
 

@@ -252,3 +252,53 @@ def test_quant_error_scale_on_tiny_workload():
     f64, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows)
     rel = np.linalg.norm(f64 - ex) / np.linalg.norm(ex)
     assert 1e-3 < rel < 0.1, rel
+
+
+# --------------------------------------------------------------------------- K-residual mode
+# ("ComfyUI-sol-attn", 核心亮点 item 1: only the residual of K inside each
+# block is quantized; the block-mean term keeps bf16 precision)
+
+def test_kres_with_error_sources_off_equals_exact():
+    """q.k = q.mean_b + q.(k - mean_b) exactly, so with every rounding switched
+    off the K-residual mode must give exact attention."""
+    w = tiny_custom(1, 2, 300, 64, seed=91, bias_sigma=4.0, outlier_frac=0.02)
+    q, k, v, _ = make_qkv(w)
+    rows = np.arange(0, 300, 7).astype(np.int32)
+    ex = oracle.attn_exact(q, k, v, w.sm_scale, rows=rows)
+    o, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows, int8_qk=False, fp8_p=False, fp8_v=False,
+                             round_bf16=False, k_residual=True)
+    assert np.max(np.abs(o - ex)) < 1e-12
+
+
+def test_kres_codes_match_numpy_restatement():
+    w = tiny_custom(1, 1, 200, 64, seed=92, bias_sigma=3.0, outlier_frac=0.05)
+    _, k, _, _ = make_qkv(w)
+    got = oracle.quantize_kres(k)
+    kf = k[0, 0].float().numpy()
+    for b in range(-(-200 // 64)):
+        blk = kf[b * 64:(b + 1) * 64].astype(np.float64)
+        mean = blk.mean(axis=0)
+        mb = torch.from_numpy(got["k_bmean"][0, 0, b].astype(np.int16)).view(torch.bfloat16).float().numpy()
+        # the stored mean is the bf16 nearest the fp64 mean (within half a bf16 step)
+        step = np.exp2(np.floor(np.log2(np.maximum(np.abs(mean), 1e-30))) - 7)
+        assert np.all(np.abs(mb.astype(np.float64) - mean) <= step / 2 + 1e-30)
+        r = (kf[b * 64:(b + 1) * 64] - mb).astype(np.float32)     # exact in fp32
+        amax = np.float32(np.abs(r).max())
+        inv = np.float32(127.0) / amax
+        want = np.clip(np.rint((r * inv).astype(np.float32)), -127, 127).astype(np.int8)
+        assert np.array_equal(got["k_i8"][0, 0, b * 64:(b + 1) * 64], want)
+        assert got["k_scale"][0, 0, b] == np.float32(amax / np.float32(127.0))
+
+
+def test_kres_block_mean_term_varies_by_block():
+    """The block-mean term must enter the scores: dropping it (a per-row constant
+    only for the global mean) would change the result."""
+    w = tiny_custom(1, 1, 256, 64, seed=93, bias_sigma=2.0)
+    q, k, v, _ = make_qkv(w)
+    k = k.clone()
+    k[0, 0, 128:] += 2.0          # a block-wise shift of the keys
+    rows = np.arange(0, 256, 5).astype(np.int32)
+    ex = oracle.attn_exact(q, k, v, w.sm_scale, rows=rows)
+    o, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows, fp8_p=False, fp8_v=False, round_bf16=False,
+                             k_residual=True)
+    assert np.linalg.norm(o - ex) / np.linalg.norm(ex) < 0.03
