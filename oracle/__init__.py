@@ -30,6 +30,7 @@ _CFLAGS = ["-O2", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off",
 
 Q_BLOCK = 128
 K_BLOCK = 64
+SEL_TILE = 128  # query / key tile of the block-sparse selection (reading S1)
 
 
 def build(force: bool = False) -> str:
@@ -58,13 +59,17 @@ def lib():
         L.oracle_quantize.argtypes = [P, I64, P, I64, P, I64, I32, I32, I32, P, P, P, P, P, P, P]
         L.oracle_attn_quant.argtypes = [P, I64, P, I64, P, I64, I32, I32, ctypes.c_float,
                                         ctypes.POINTER(_Flags), P, I32, P, P]
+        L.oracle_attn_quant_masked.argtypes = [P, I64, P, I64, P, I64, I32, I32, ctypes.c_float,
+                                               ctypes.POINTER(_Flags), P, P, I32, P, P]
+        L.oracle_block_scores.argtypes = [P, P, P, P, I32, I32, ctypes.c_float, P]
+        L.oracle_block_select.argtypes = [P, I32, ctypes.c_double, P]
         L.oracle_int8_gemm_nt.argtypes = [P, I64, P, I64, I32, I32, I32, P]
         L.oracle_quantize_kres.argtypes = [P, I64, I32, I32, P, P, P]
         L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         L.oracle_e4m3_decode_array.argtypes = [P, I64, P]
         L.oracle_bf16_rne_array.argtypes = [P, I64, P]
         for f in ("oracle_attn_exact", "oracle_quantize", "oracle_attn_quant", "oracle_int8_gemm_nt",
-                  "oracle_quantize_kres"):
+                  "oracle_quantize_kres", "oracle_attn_quant_masked", "oracle_block_scores", "oracle_block_select"):
             getattr(L, f).restype = I32
         _lib = L
     return _lib
@@ -167,13 +172,20 @@ def quantize_kres(k):
 
 
 def attn_quant(q, k, v, sm_scale, rows=None, int8_qk=True, fp8_p=True, fp8_v=True,
-               round_bf16=True, smooth_k=True, heads=None, k_residual=False):
+               round_bf16=True, smooth_k=True, heads=None, k_residual=False, kv_keep=None):
     """Quant-emulation attention.  Returns (out_f64 [B,H,R,d], out_bf16 bits [B,H,R,d] uint16).
     ``heads`` optionally restricts the work to a list of (b, h) pairs (others stay zero).
     ``k_residual``: K-residual quantization with the block-mean term kept
-    (oracle_quantize_kres) instead of the smoothing."""
+    (oracle_quantize_kres) instead of the smoothing.
+    ``kv_keep``: block-sparse skipping, [B,H,nt,nt] (nt = ceil(N/128)), nonzero
+    where query tile i attends to key tile j; a row whose tile keeps nothing
+    returns 0 (oracle_attn_quant_masked)."""
     B, H, N, d = q.shape
     r = _rows_array(rows, N)
+    nt = -(-N // SEL_TILE)
+    if kv_keep is not None:
+        kv_keep = np.asarray(kv_keep)
+        assert kv_keep.shape == (B, H, nt, nt), kv_keep.shape
     f = _Flags(int(int8_qk), int(fp8_p), int(fp8_v), int(round_bf16), int(smooth_k), int(k_residual))
     out = np.zeros((B, H, len(r), d), dtype=np.float64)
     outb = np.zeros((B, H, len(r), d), dtype=np.uint16)
@@ -183,11 +195,63 @@ def attn_quant(q, k, v, sm_scale, rows=None, int8_qk=True, fp8_p=True, fp8_v=Tru
         (qp, qs), (kp, ks), (vp, vs) = _slab(q, b, h), _slab(k, b, h), _slab(v, b, h)
         ob = np.zeros((len(r), d), dtype=np.float64)
         obb = np.zeros((len(r), d), dtype=np.uint16)
-        _check(L.oracle_attn_quant(qp, qs, kp, ks, vp, vs, N, d, ctypes.c_float(sm_scale),
-                                   ctypes.byref(f), _ptr(r), len(r), _ptr(ob), _ptr(obb)), "attn_quant")
+        keep = None if kv_keep is None else np.ascontiguousarray(kv_keep[b, h] != 0, dtype=np.uint8)
+        _check(L.oracle_attn_quant_masked(qp, qs, kp, ks, vp, vs, N, d, ctypes.c_float(sm_scale),
+                                          ctypes.byref(f), _ptr(keep) if keep is not None else None,
+                                          _ptr(r), len(r), _ptr(ob), _ptr(obb)), "attn_quant")
         out[b, h] = ob
         outb[b, h] = obb
     return out, outb
+
+
+def block_scores(q, k, v, sm_scale, codes=None):
+    """Tile-pair scores of the block-sparse selection (reading S2,
+    oracle_block_scores): [B,H,nt,nt] float32, from the oracle's own codes
+    (``codes`` = a result of quantize(q, k, v), computed if not given)."""
+    B, H, N, d = q.shape
+    nt = -(-N // SEL_TILE)
+    c = quantize(q, k, v) if codes is None else codes
+    out = np.zeros((B, H, nt, nt), dtype=np.float32)
+    L = lib()
+    for b in range(B):
+        for h in range(H):
+            qc = np.ascontiguousarray(c["q_i8"][b, h])
+            kc = np.ascontiguousarray(c["k_i8"][b, h])
+            qs = np.ascontiguousarray(c["q_scale"][b, h], dtype=np.float32)
+            ks = np.ascontiguousarray(c["k_scale"][b, h], dtype=np.float32)
+            sb = np.zeros((nt, nt), dtype=np.float32)
+            _check(L.oracle_block_scores(_ptr(qc), _ptr(qs), _ptr(kc), _ptr(ks), N, d,
+                                         ctypes.c_float(sm_scale), _ptr(sb)), "block_scores")
+            out[b, h] = sb
+    return out
+
+
+def block_select(sbar, N, tau):
+    """Kept key tiles per query tile (reading S3, oracle_block_select):
+    uint8 [B,H,nt,nt] from scores [B,H,nt,nt]."""
+    sbar = np.asarray(sbar, dtype=np.float32)
+    B, H, nt, _ = sbar.shape
+    assert nt == -(-N // SEL_TILE)
+    keep = np.zeros((B, H, nt, nt), dtype=np.uint8)
+    L = lib()
+    for b in range(B):
+        for h in range(H):
+            sb = np.ascontiguousarray(sbar[b, h])
+            kb = np.zeros((nt, nt), dtype=np.uint8)
+            _check(L.oracle_block_select(_ptr(sb), N, float(tau), _ptr(kb)), "block_select")
+            keep[b, h] = kb
+    return keep
+
+
+def tau_schedule(step, n_steps, tau_start, tau_end):
+    """Reading S4: tau at sampling step ``step`` of ``n_steps``, moving linearly
+    from tau_start (first step) to tau_end (last step); steps outside the
+    range take the nearer end ("ComfyUI-sol-attn", 核心亮点 item 4: sparse
+    early, dense late)."""
+    if n_steps <= 1:
+        return float(tau_end)
+    t = min(max(step, 0), n_steps - 1) / (n_steps - 1)
+    return float(tau_start) + (float(tau_end) - float(tau_start)) * t
 
 
 def int8_gemm_nt(a: np.ndarray, b: np.ndarray) -> np.ndarray:

@@ -31,6 +31,10 @@
  *   核心亮点 item 1 instead of the smoothing: only the residual of K inside
  *   each 64-token block is quantized, and the block mean term stays at bf16
  *   precision -- see oracle_quantize_kres.)
+ *   oracle_attn_quant_masked -- the same with block-sparse skipping: each
+ *                         128-query tile attends only to the 128-key tiles
+ *                         its row of a keep mask selects (see the block
+ *                         selection below for how such a mask is chosen).
  *   oracle_attn_quant  -- the quantization scheme, step by step, in the order
  *                         smoothing -> block INT8 of Q and K -> integer Q K^T ->
  *                         dequant -> softmax with an integer-grid (log2) row max
@@ -51,6 +55,11 @@
  *                      block codes against closed forms; the one-pass
  *                      integer-grid softmax against a tile-by-tile replay of
  *                      the online algorithm.
+ *   block sparsity  -- tile scores against the mean of the fp64 dequantized
+ *                      score matrix; the kept sets against the properties
+ *                      that define reading S3 (ranking prefix, mass reaches
+ *                      tau, no redundant tile, nested in tau); masked exact
+ *                      mode against a brute-force softmax over the kept keys.
  *
  * Build:  gcc -O2 -std=c11 -fPIC -shared -ffp-contract=off -fno-fast-math
  *             -fexcess-precision=standard -o liboracle.so sage_oracle.c -lm
@@ -64,6 +73,7 @@
 #define ORACLE_Q_BLOCK 128 /* Q tokens per quantization block (reading C3) */
 #define ORACLE_K_BLOCK 64  /* K tokens per quantization block (reading C3) */
 #define ORACLE_E4M3_MAX 448.0
+#define ORACLE_SEL_TILE 128 /* tokens per query / key tile of the block selection (reading S1) */
 
 /* ------------------------------------------------------------------------ */
 /* Number formats                                                           */
@@ -386,14 +396,19 @@ typedef struct {
  * out_f64 (may be NULL) receives the value before the bf16 rounding,
  * out_bf16 (may be NULL) the rounded bit pattern; both [nrows][d].
  */
-int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
-                      const uint16_t *k, int64_t k_rs,
-                      const uint16_t *v, int64_t v_rs,
-                      int N, int d, float sm_scale,
-                      const oracle_quant_flags *flags,
-                      const int32_t *rows, int nrows,
-                      double *out_f64, uint16_t *out_bf16)
+int oracle_attn_quant_masked(const uint16_t *q, int64_t q_rs,
+                             const uint16_t *k, int64_t k_rs,
+                             const uint16_t *v, int64_t v_rs,
+                             int N, int d, float sm_scale,
+                             const oracle_quant_flags *flags,
+                             const uint8_t *keep,
+                             const int32_t *rows, int nrows,
+                             double *out_f64, uint16_t *out_bf16)
 {
+    /* keep (may be NULL = every key): [nt][nt] with nt = ceil(N/128); key j
+     * takes part in row r's softmax iff keep[(r/128)*nt + j/128] != 0.  A row
+     * whose tile keeps no key tile has no softmax: its output is 0. */
+    const int nt = (N + ORACLE_SEL_TILE - 1) / ORACLE_SEL_TILE;
     if (N <= 0 || d <= 0 || !flags) return -1;
     int nqb = (N + ORACLE_Q_BLOCK - 1) / ORACLE_Q_BLOCK;
     int nkb = (N + ORACLE_K_BLOCK - 1) / ORACLE_K_BLOCK;
@@ -439,7 +454,12 @@ int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
                            oracle_bf16_to_double(kbm[(size_t)b * d + c]);
             e[b] = acc * (double)sm_scale * 1.4426950408889634;
         }
+        const uint8_t *krow = keep ? keep + (size_t)(r / ORACLE_SEL_TILE) * nt : NULL;
         for (int j = 0; j < N; ++j) {
+            if (krow && !krow[j / ORACLE_SEL_TILE]) {
+                x[j] = -INFINITY; /* skipped key tile */
+                continue;
+            }
             if (flags->int8_qk) {
                 int64_t S = 0;
                 for (int c = 0; c < d; ++c)
@@ -458,6 +478,13 @@ int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
                 x[j] = acc * (double)sm_scale * 1.4426950408889634 + e[j / ORACLE_K_BLOCK];
             }
             if (x[j] > xmax) xmax = x[j];
+        }
+        if (xmax == -INFINITY) { /* no key kept */
+            for (int c = 0; c < d; ++c) {
+                if (out_f64) out_f64[(size_t)ri * d + c] = 0.0;
+                if (out_bf16) out_bf16[(size_t)ri * d + c] = 0;
+            }
+            continue;
         }
         double m = ceil(xmax);
         double l = 0.0;
@@ -479,6 +506,134 @@ done:
     free(qc); free(kc); free(vc); free(qs); free(ks); free(km); free(vs);
     free(x); free(vval); free(o); free(kbm); free(e);
     return rc;
+}
+
+int oracle_attn_quant(const uint16_t *q, int64_t q_rs,
+                      const uint16_t *k, int64_t k_rs,
+                      const uint16_t *v, int64_t v_rs,
+                      int N, int d, float sm_scale,
+                      const oracle_quant_flags *flags,
+                      const int32_t *rows, int nrows,
+                      double *out_f64, uint16_t *out_bf16)
+{
+    return oracle_attn_quant_masked(q, q_rs, k, k_rs, v, v_rs, N, d, sm_scale, flags, NULL, rows, nrows,
+                                    out_f64, out_bf16);
+}
+
+/* ------------------------------------------------------------------------ */
+/* Block-sparse skipping ("ComfyUI-sol-attn", 核心亮点 item 4 and its node   */
+/* table: a sparsity value tau that may ramp over the sampling steps, sparse */
+/* early and dense late).  The page names the control only; the readings    */
+/* S1-S4 below are this project's.                                          */
+/* ------------------------------------------------------------------------ */
+
+/* Reading S1/S2 -- tiles and their score.  Queries and keys are cut into
+ * tiles of 128 tokens (the Q quantization block; two K blocks).  The score of
+ * (query tile i, key tile j) is the mean of the dequantized scores x_rs over
+ * the tile pair, in log2 units:
+ *     sbar_ij = (sum_r q_r) . (sum_s k_s) * fp32(sm_scale*log2 e) / (n_i n_j)
+ * with q_r = q_scale(r) * qcode_r, k_s = k_scale(s) * kcode_s.  It is
+ * computed in IEEE fp32 in this exact order, one rounding per operation:
+ *     qs_i[c] = q_scale[i] * float(sum of Q codes of tile i, channel c)
+ *     ks_j[c] = k_scale[2j] * float(sum over K block 2j)
+ *             + k_scale[2j+1] * float(sum over K block 2j+1)
+ *     dot     = (((0 + qs[0] ks[0]) + qs[1] ks[1]) + ...)     (c ascending)
+ *     sbar    = (dot * s_l2) / float(n_i * n_j)
+ * (the code sums are exact integers, so everything before the first fp32
+ * product is order-independent).  Padded tokens (n >= N) take no part.
+ * sbar is [nt][nt] row-major; q_scale has ceil(N/128) and k_scale ceil(N/64)
+ * entries. */
+int oracle_block_scores(const int8_t *qc, const float *qs, const int8_t *kc, const float *ks,
+                        int N, int d, float sm_scale, float *sbar)
+{
+    if (N <= 0 || d <= 0) return -1;
+    const int nt = (N + ORACLE_SEL_TILE - 1) / ORACLE_SEL_TILE;
+    const int nkb = (N + ORACLE_K_BLOCK - 1) / ORACLE_K_BLOCK;
+    float *qv = (float *)malloc(sizeof(float) * (size_t)nt * d);
+    float *kv = (float *)malloc(sizeof(float) * (size_t)nt * d);
+    if (!qv || !kv) { free(qv); free(kv); return -2; }
+    for (int i = 0; i < nt; ++i) {
+        const int r0 = i * ORACLE_SEL_TILE;
+        for (int c = 0; c < d; ++c) {
+            int64_t sq = 0, sa = 0, sb = 0;
+            for (int r = r0; r < r0 + ORACLE_SEL_TILE && r < N; ++r) {
+                sq += qc[(size_t)r * d + c];
+                if (r < r0 + ORACLE_K_BLOCK) sa += kc[(size_t)r * d + c];
+                else sb += kc[(size_t)r * d + c];
+            }
+            qv[(size_t)i * d + c] = qs[i] * (float)sq;
+            const float kb0 = ks[2 * i] * (float)sa;
+            const float kb1 = (2 * i + 1 < nkb ? ks[2 * i + 1] : 0.f) * (float)sb;
+            kv[(size_t)i * d + c] = kb0 + kb1;
+        }
+    }
+    const float s_l2 = sm_scale * (float)1.4426950408889634;
+    for (int i = 0; i < nt; ++i) {
+        const int ni = (N - i * ORACLE_SEL_TILE) < ORACLE_SEL_TILE ? N - i * ORACLE_SEL_TILE : ORACLE_SEL_TILE;
+        for (int j = 0; j < nt; ++j) {
+            const int nj = (N - j * ORACLE_SEL_TILE) < ORACLE_SEL_TILE ? N - j * ORACLE_SEL_TILE : ORACLE_SEL_TILE;
+            float dot = 0.f;
+            for (int c = 0; c < d; ++c) {
+                const float prod = qv[(size_t)i * d + c] * kv[(size_t)j * d + c];
+                dot = dot + prod;
+            }
+            const float num = dot * s_l2;
+            sbar[(size_t)i * nt + j] = num / (float)(ni * nj);
+        }
+    }
+    free(qv);
+    free(kv);
+    return 0;
+}
+
+/* Reading S3 -- which key tiles a query tile keeps.  The estimated softmax
+ * mass of key tile j for query tile i is w_ij = n_j * 2^(sbar_ij - max_j
+ * sbar_ij) (fp64 here).  The key tiles are ranked by sbar descending, ties by
+ * the lower index; the tile at rank t is kept iff the mass of the tiles ranked
+ * before it is below tau times the total mass.  So the kept set is the
+ * shortest prefix of the ranking whose mass reaches tau of the total; it is
+ * never empty, and tau >= 1 keeps every tile.  keep is [nt][nt] (1 = kept). */
+int oracle_block_select(const float *sbar, int N, double tau, uint8_t *keep)
+{
+    if (N <= 0 || !(tau > 0.0)) return -1;
+    const int nt = (N + ORACLE_SEL_TILE - 1) / ORACLE_SEL_TILE;
+    int *order = (int *)malloc(sizeof(int) * (size_t)nt);
+    double *w = (double *)malloc(sizeof(double) * (size_t)nt);
+    if (!order || !w) { free(order); free(w); return -2; }
+    for (int i = 0; i < nt; ++i) {
+        const float *row = sbar + (size_t)i * nt;
+        uint8_t *kr = keep + (size_t)i * nt;
+        if (tau >= 1.0) {
+            for (int j = 0; j < nt; ++j) kr[j] = 1;
+            continue;
+        }
+        /* insertion sort: sbar descending, index ascending on ties */
+        for (int j = 0; j < nt; ++j) {
+            int t = j;
+            while (t > 0 && (row[order[t - 1]] < row[j] || (row[order[t - 1]] == row[j] && order[t - 1] > j))) {
+                order[t] = order[t - 1];
+                --t;
+            }
+            order[t] = j;
+        }
+        const double top = (double)row[order[0]];
+        double total = 0.0;
+        for (int t = 0; t < nt; ++t) {
+            const int j = order[t];
+            const int nj = (N - j * ORACLE_SEL_TILE) < ORACLE_SEL_TILE ? N - j * ORACLE_SEL_TILE : ORACLE_SEL_TILE;
+            w[t] = (double)nj * exp2((double)row[j] - top);
+            total += w[t];
+        }
+        for (int j = 0; j < nt; ++j) kr[j] = 0;
+        double before = 0.0;
+        for (int t = 0; t < nt && before < tau * total; ++t) {
+            kr[order[t]] = 1;
+            before += w[t];
+        }
+    }
+    free(order);
+    free(w);
+    return 0;
 }
 
 /* Integer score tile from given codes: s[i][j] = sum_c a[i][c] * b[j][c]
