@@ -33,7 +33,7 @@ METRIC = "quantized attention TOPS (4·B·H·N²·d/t) and ms/call at N=4608 and
 DTYPE = "i8/e4m3"        # QK^T on int8 codes, PV on e4m3 codes; bf16 in and out
 PRIMARY, SECONDARY = "flux", "video"
 PEAK_NOTE = "measured cuBLAS bf16 burst x 2 (nominal 8-bit/bf16 dense ratio)"
-LAUNCHES_PER_STEP = 4    # stats partial, stats final, quantize, attention
+LAUNCHES_PER_STEP = 3    # k_stats (partial K/V statistics), k_quant (finishes them, codes), k_attn
 
 
 def _env_int(name, default):
@@ -195,14 +195,24 @@ def run_gpu(args):
     def measure(w, steps, warmup):
         q, k, v, bufs = make_qkv(w, device=dev)
         out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
-        ws = torch.empty(sage.sage_attn_workspace_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
+        sparse = args.tau is not None
+        ws_bytes = (sage.sage_attn_sparse_workspace_bytes if sparse else sage.sage_attn_workspace_bytes)(
+            w.B, w.H, w.N, w.d)
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+
+        def forward(events=None):
+            if sparse:
+                return sage.sage_attn_fwd_sparse(q, k, v, tau=args.tau, sm_scale=w.sm_scale, out=out, workspace=ws,
+                                                 attn_events=events)
+            return sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws, attn_events=events)
+
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
         for e in ev:
             for x in e:
                 x.record()          # create the underlying events
         for _ in range(warmup):
-            sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws)
+            forward()
         torch.cuda.synchronize()
         sage.sage_check()
         barrier()
@@ -213,7 +223,7 @@ def run_gpu(args):
             flush.zero_()
             s0, a0, a1, s1 = ev[i]
             s0.record()
-            sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws, attn_events=(a0, a1))
+            forward((a0, a1))
             s1.record()
         torch.cuda.synchronize()
         barrier()
@@ -224,6 +234,11 @@ def run_gpu(args):
         attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
         total_ms = max_over_ranks(sum(step_ms))
         attn_avg = max_over_ranks(sum(attn_ms) / steps)
+        kept = 1.0
+        if sparse:  # fraction of (query tile, key tile) pairs the selection kept, outside the timed region
+            _, mask = sage.sage_attn_fwd_sparse(q, k, v, tau=args.tau, sm_scale=w.sm_scale, out=out, workspace=ws,
+                                                return_mask=True)
+            kept = float(sage.mask_to_keep(mask, sage.n_tiles(w.N)).float().mean().item())
         # end to end through host memory: pinned input -> device, forward, result -> pinned host
         host_in = bufs[0].cpu().pin_memory() if w.layout == "fused" else torch.stack(bufs).cpu().pin_memory()
         ws_host = torch.empty(sage.sage_attn_fwd_host_scratch_bytes(w.B, w.H, w.N, w.d), dtype=torch.uint8, device=dev)
@@ -247,13 +262,13 @@ def run_gpu(args):
         d2h = out_host.numel() * out_host.element_size()
         del q, k, v, bufs, out, ws, host_in, ws_host
         torch.cuda.empty_cache()
-        return dict(total_ms=total_ms, attn_ms=attn_avg, e2e_ms=e2e_ms, clocks=clocks, h2d=h2d, d2h=d2h)
+        return dict(total_ms=total_ms, attn_ms=attn_avg, e2e_ms=e2e_ms, clocks=clocks, h2d=h2d, d2h=d2h, kept=kept)
 
     wp = WORKLOADS[args.workload]
     r = measure(wp, args.steps, args.warmup)
     ms = r["total_ms"] / args.steps
     value = whole_job_tops(world, wp.ops, args.steps, r["total_ms"])
-    attn_tops = wp.ops / (r["attn_ms"] * 1e-3) / 1e12
+    attn_tops = r["kept"] * wp.ops / (r["attn_ms"] * 1e-3) / 1e12  # the kernel's own work
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -263,15 +278,22 @@ def run_gpu(args):
                    "l2": "flushed before every timed step (256 MB write, outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "k_attn (fused attention)", "achieved": round(attn_tops, 2),
                      "peak": round(peak_8bit, 1), "unit": "TFLOP/s", "frac": round(attn_tops / peak_8bit, 4),
-                     "traffic": _attn_traffic(wp.name), "peak_source": f"{peak_kind}: {PEAK_NOTE}",
+                     "traffic": None if args.tau is not None else _attn_traffic(wp.name),
+                     "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
-                "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on two streams, quantize + attention, bf16 out -> pinned host)"},
-        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+                "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
+                       "attention, bf16 out -> pinned host; dense)"},
+        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.tau is not None and args.tau < 1 else 0)) * args.steps,
         "clocks": r["clocks"],
     }
-    if args.secondary and args.workload != SECONDARY:
+    if args.tau is not None:
+        line["config"]["tau"] = args.tau
+        line["config"]["kept_fraction"] = round(r["kept"], 4)
+        line["config"]["ops"] = ("value counts the dense 4*B*H*N^2*d; roofline.achieved counts the kept tile "
+                                 "pairs only (block-sparse forward, sage_attn_fwd_sparse)")
+    if args.secondary and args.workload != SECONDARY and args.tau is None:
         ws_ = WORKLOADS[SECONDARY]
         r2 = measure(ws_, max(3, args.steps // 2), args.warmup)
         k2 = max(3, args.steps // 2)
@@ -330,6 +352,8 @@ def main():
     ap.add_argument("--no-secondary", dest="secondary", action="store_false")
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--tau", type=float, default=None,
+                    help="time the block-sparse forward with this tau instead of the dense one")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

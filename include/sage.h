@@ -23,7 +23,8 @@
  *          block-wise computation that never writes the attention matrix out.
  *   [SOL]  "ComfyUI-sol-attn" page, "核心亮点" items 2 and 4: zero-copy reads of a
  *          fused-qkv strided view; explicit, logged rejection of unsupported
- *          inputs instead of a silent fallback.
+ *          inputs instead of a silent fallback; scheduled sparsity, a value
+ *          tau that may ramp over the sampling steps (sparse early, dense late).
  * Numeric points the pages leave open follow the readings C1..C9 of the
  * project's design notes (block sizes, rounding modes, integer-grid row max,
  * 448 P scale, per-channel V scale, fp32 accumulation, bf16 RNE output).
@@ -212,8 +213,8 @@ size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d);
  * sage_attn_fwd_host -- sage_attn_fwd on HOST memory, the end-to-end call:
  * `qkv_host` (bf16, `layout` as above) goes to the device, the forward runs,
  * and the bf16 result lands in `out_host` ([B,H,N,d] contiguous).  The heads
- * are processed in chunks on two internal streams so that host<->device
- * copies overlap the kernels of the other chunk; each chunk's result is the
+ * are processed in chunks on three internal streams so that host<->device
+ * copies overlap the kernels of other chunks; each chunk's result is the
  * whole call's result for its heads, bit for bit (every statistic is per
  * head).  Host buffers should be page-locked (cudaHostAlloc / pinned) for the
  * copies to be asynchronous; pageable buffers work but serialise.
@@ -229,6 +230,80 @@ size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d);
 sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_host,
                                  int B, int H, int N, int d, float sm_scale,
                                  void *scratch, size_t scratch_bytes, sage_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Block-sparse skipping ([SOL] item 4).  The page names only the control     */
+/* (tau, ramped over the sampling steps); the steps are this library's        */
+/* readings S1-S4:                                                           */
+/*   S1 query and key tiles of 128 tokens;                                    */
+/*   S2 tile-pair score = mean dequantized score of the pair in log2 units,   */
+/*      (sum_i q).(sum_j k) * fp32(sm_scale*log2 e) / (n_i n_j), from the    */
+/*      codes of sage_quant_qk, in fp32 in a fixed order;                     */
+/*   S3 query tile i keeps the shortest prefix of its key tiles, ranked by    */
+/*      score (ties: lower index first), whose estimated mass                 */
+/*      n_j 2^(score - top score) reaches tau of the row's total; tau >= 1    */
+/*      keeps every tile, and a row never keeps fewer than one;               */
+/*   S4 sage_tau_schedule: tau moves linearly over the sampling steps.        */
+/* Mask layout: uint32 words [B*H][T][W], T = ceil(N/128) tiles,              */
+/* W = ceil(T/32); bit j of row (b*H+h, i) set = query tile i attends to key  */
+/* tile j.  A query tile whose row is empty gets output 0.  Sparse calls      */
+/* accept N up to 4096*128 tokens (T <= 4096); larger is SAGE_ERR_UNSUPPORTED.*/
+/* ------------------------------------------------------------------------ */
+
+/* Bytes of one mask (0 for a shape rejected): B*H*T*W*4. */
+size_t sage_block_mask_bytes(int B, int H, int N);
+
+/* Bytes of scratch sage_block_select needs (0 for a shape rejected). */
+size_t sage_block_select_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * sage_block_select -- readings S2 and S3 on the codes of sage_quant_qk
+ * (q_i8/k_i8 [B,H,N_pad,d], q_scale [B,H,N_pad/128], k_scale [B,H,N_pad/64]):
+ * writes `mask` (device, 4-byte aligned, sage_block_mask_bytes) and, if
+ * `scores` is not NULL, the tile-pair scores as fp32 [B*H][T][T].
+ * tau must be finite and > 0.  workspace: >= sage_block_select_workspace_bytes
+ * bytes, 256-byte aligned, or NULL (stream-ordered allocation).
+ */
+sage_status_t sage_block_select(const int8_t *q_i8, const float *q_scale,
+                                const int8_t *k_i8, const float *k_scale,
+                                int B, int H, int N, int d, float sm_scale, float tau,
+                                uint32_t *mask, float *scores,
+                                void *workspace, size_t workspace_bytes,
+                                sage_stream_t stream);
+
+/* Bytes of scratch sage_attn_fwd_sparse needs: the forward's plus the
+ * selection's plus one mask. */
+size_t sage_attn_sparse_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * sage_attn_fwd_sparse -- sage_attn_fwd with block-sparse skipping: the
+ * quantize pass, then the key-tile mask (mask_in if not NULL, else
+ * sage_block_select with `tau`, copied to mask_out if that is not NULL), then
+ * the fused attention kernel visiting only each query tile's kept key tiles.
+ * With every bit set the result equals sage_attn_fwd's bit for bit; with
+ * tau >= 1 and no mask_in the dense kernel runs (the same result).
+ * attn_begin / attn_end: optional events recorded around the attention kernel
+ * (as in sage_attn_fwd_ev).  Errors as sage_attn_fwd, plus SAGE_ERR_INVALID_ARG
+ * for tau (when no mask_in is given) and misaligned masks, and
+ * SAGE_ERR_UNSUPPORTED for T > 4096.
+ */
+sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4],
+                                   const void *k, const int64_t k_stride[4],
+                                   const void *v, const int64_t v_stride[4],
+                                   void *out, const int64_t o_stride[4],
+                                   int B, int H, int N, int d, float sm_scale, float tau,
+                                   const uint32_t *mask_in, uint32_t *mask_out,
+                                   void *workspace, size_t workspace_bytes,
+                                   sage_stream_t stream,
+                                   sage_event_t attn_begin, sage_event_t attn_end);
+
+/*
+ * sage_tau_schedule -- reading S4: tau at sampling step `step` of `n_steps`,
+ * tau_start at the first step moving linearly to tau_end at the last (steps
+ * outside the range clamp to it; one step gives tau_end).  [SOL] item 4 ramps
+ * from sparse (small tau) early to dense (tau = 1) late.  Host function.
+ */
+float sage_tau_schedule(int step, int n_steps, float tau_start, float tau_end);
 
 /*
  * sage_attn_dense_ref_gpu -- plain dense attention on the CUDA cores in fp32

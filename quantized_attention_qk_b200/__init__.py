@@ -21,6 +21,8 @@ __all__ = [
     "SageError", "lib", "sage_attn_fwd", "sage_attn_quantized", "sage_quant_qk", "sage_quant_v",
     "sage_attn_dense_ref_gpu", "sage_debug_qk_tile", "sage_quant_qk_noalloc", "sage_attn_workspace_bytes",
     "sage_quant_workspace_bytes", "sage_check", "sage_attn_fwd_host", "n_pad",
+    "sage_block_select", "sage_attn_fwd_sparse", "sage_tau_schedule", "sage_block_mask_bytes",
+    "sage_attn_sparse_workspace_bytes", "n_tiles", "mask_words", "mask_to_keep", "keep_to_mask",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -58,6 +60,14 @@ _SIGS = {
     "sage_debug_qk_tile": ([_P, _P, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _I32, _P, _P], _I32),
     "sage_attn_fwd_host_scratch_bytes": ([_I32, _I32, _I32, _I32], _SZ),
     "sage_attn_fwd_host": ([_P, _I32, _P, _I32, _I32, _I32, _I32, ctypes.c_float, _P, _SZ, _P], _I32),
+    "sage_block_mask_bytes": ([_I32, _I32, _I32], _SZ),
+    "sage_block_select_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_block_select": ([_P, _P, _P, _P, _I32, _I32, _I32, _I32, ctypes.c_float, ctypes.c_float, _P, _P, _P, _SZ,
+                           _P], _I32),
+    "sage_attn_sparse_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_attn_fwd_sparse": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                              ctypes.c_float, _P, _P, _P, _SZ, _P, _P, _P], _I32),
+    "sage_tau_schedule": ([_I32, _I32, ctypes.c_float, ctypes.c_float], ctypes.c_float),
 }
 
 
@@ -271,3 +281,94 @@ def sage_attn_fwd_host(qkv_host, B, H, N, d, layout="fused", sm_scale=None, devi
         _raise(lib().sage_attn_fwd_host(_ptr(qkv_host), LAYOUTS[layout], _ptr(out_host), B, H, N, d,
                                         ctypes.c_float(sm_scale), _ptr(workspace), ws_bytes, _stream(stream, dev)))
     return out_host
+
+
+# --------------------------------------------------------------------------
+# block-sparse skipping (readings S1-S4 of the sol-attn page's scheduled
+# sparsity; the layout of a mask is described in include/sage.h)
+# --------------------------------------------------------------------------
+
+TILE = 128  # query / key tile of the block-sparse mask
+
+
+def n_tiles(N: int) -> int:
+    return -(-N // TILE)
+
+
+def mask_words(N: int) -> int:
+    return -(-n_tiles(N) // 32)
+
+
+def sage_block_mask_bytes(B: int, H: int, N: int) -> int:
+    return int(lib().sage_block_mask_bytes(B, H, N))
+
+
+def sage_attn_sparse_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().sage_attn_sparse_workspace_bytes(B, H, N, d))
+
+
+def sage_tau_schedule(step: int, n_steps: int, tau_start: float, tau_end: float) -> float:
+    return float(lib().sage_tau_schedule(step, n_steps, ctypes.c_float(tau_start), ctypes.c_float(tau_end)))
+
+
+def keep_to_mask(keep: torch.Tensor) -> torch.Tensor:
+    """[B,H,T,T] bool/int (nonzero = query tile i keeps key tile j) -> int32
+    mask words [B,H,T,W] in the library's layout (bit j % 32 of word j // 32).
+    Argument marshalling only: packs bits, on the tensor's device."""
+    B, H, T, T2 = keep.shape
+    assert T == T2
+    W = -(-T // 32)
+    k = torch.zeros(B, H, T, W * 32, dtype=torch.int64, device=keep.device)
+    k[..., :T] = (keep != 0).to(torch.int64)
+    weights = (torch.ones(32, dtype=torch.int64, device=keep.device) << torch.arange(32, device=keep.device))
+    words = (k.view(B, H, T, W, 32) * weights).sum(-1)
+    return torch.where(words >= 2 ** 31, words - 2 ** 32, words).to(torch.int32)
+
+
+def mask_to_keep(mask: torch.Tensor, T: int) -> torch.Tensor:
+    """int32 mask words [B,H,T,W] -> bool [B,H,T,T] (the inverse of keep_to_mask)."""
+    m = mask.to(torch.int64) & 0xFFFFFFFF
+    bits = (m.unsqueeze(-1) >> torch.arange(32, device=mask.device)) & 1
+    return bits.flatten(-2)[..., :T].bool()
+
+
+def sage_block_select(codes, N: int, sm_scale: float, tau: float, want_scores=False, workspace=None, stream=None):
+    """Key-tile mask of every query tile from the codes of sage_quant_qk
+    (readings S2, S3).  Returns int32 mask words [B,H,T,W] (and the fp32 tile
+    scores [B,H,T,T] with want_scores)."""
+    q_i8, k_i8 = codes["q_i8"], codes["k_i8"]
+    B, H, _, d = q_i8.shape
+    dev = q_i8.device
+    T, W = n_tiles(N), mask_words(N)
+    mask = torch.empty(B, H, T, W, dtype=torch.int32, device=dev)
+    scores = torch.empty(B, H, T, T, dtype=torch.float32, device=dev) if want_scores else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _raise(lib().sage_block_select(_ptr(q_i8), _ptr(codes["q_scale"]), _ptr(k_i8), _ptr(codes["k_scale"]),
+                                   B, H, N, d, ctypes.c_float(sm_scale), ctypes.c_float(tau), _ptr(mask),
+                                   _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream, dev)))
+    return (mask, scores) if want_scores else mask
+
+
+def sage_attn_fwd_sparse(q, k, v, tau=1.0, sm_scale=None, mask=None, return_mask=False, out=None, workspace=None,
+                         stream=None, attn_events=None):
+    """Quantized attention forward with block-sparse skipping.  ``mask``:
+    optional int32 mask words [B,H,T,W] (then ``tau`` is not used); otherwise
+    the library selects with ``tau``.  Returns out (and the mask used, with
+    return_mask)."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    dev = q.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    mask_out = None
+    if return_mask:
+        mask_out = torch.empty(B, H, n_tiles(N), mask_words(N), dtype=torch.int32, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
+    _raise(lib().sage_attn_fwd_sparse(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                      _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                      ctypes.c_float(tau), _ptr(mask), _ptr(mask_out), _ptr(workspace), ws_bytes,
+                                      _stream(stream, dev), e0, e1))
+    return (out, mask_out) if return_mask else out

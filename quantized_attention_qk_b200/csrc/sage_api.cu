@@ -299,6 +299,108 @@ sage_status_t sage_attn_fwd(const void *q, const int64_t q_stride[4], const void
                             workspace_bytes, stream, nullptr, nullptr);
 }
 
+static sage_status_t check_sparse_shape(int B, int H, int N, int d) {
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r) return r;
+    const Shape s{B, H, N, d};
+    if (s.n_tiles() > kMaxSelectTiles)
+        return fail(SAGE_ERR_UNSUPPORTED, "block-sparse calls take at most %d tiles of 128 tokens (N=%d gives %d)",
+                    kMaxSelectTiles, N, s.n_tiles());
+    return SAGE_OK;
+}
+
+static sage_status_t check_tau(float tau) {
+    if (!std::isfinite(tau) || !(tau > 0.f))
+        return fail(SAGE_ERR_INVALID_ARG, "tau=%g must be finite and > 0", (double)tau);
+    return SAGE_OK;
+}
+
+size_t sage_block_mask_bytes(int B, int H, int N) {
+    if (B < 1 || H < 1 || N < 1) return 0;
+    const Shape s{B, H, N, 128};
+    if (s.n_tiles() > kMaxSelectTiles) return 0;
+    return mask_bytes(s);
+}
+
+size_t sage_block_select_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    const Shape s{B, H, N, d};
+    if (s.n_tiles() > kMaxSelectTiles) return 0;
+    return select_ws_bytes(s);
+}
+
+sage_status_t sage_block_select(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8, const float *k_scale,
+                                int B, int H, int N, int d, float sm_scale, float tau, uint32_t *mask, float *scores,
+                                void *workspace, size_t workspace_bytes, sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_sparse_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_tau(tau)) ||
+        (r = check_dev(q_i8, "q_i8", 16)) || (r = check_dev(k_i8, "k_i8", 16)) ||
+        (r = check_dev(q_scale, "q_scale", 4)) || (r = check_dev(k_scale, "k_scale", 4)) ||
+        (r = check_dev(mask, "mask", 4)) || (scores && (r = check_dev(scores, "scores", 4))))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    if ((r = get_scratch(scr, workspace, workspace_bytes, select_ws_bytes(s), st))) return r;
+    cudaError_t e = launch_select(s, q_i8, q_scale, k_i8, k_scale, sm_scale, tau, scr.ptr, mask, scores, st);
+    if (e != cudaSuccess) return cuda_fail(e, "block selection");
+    return SAGE_OK;
+}
+
+size_t sage_attn_sparse_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    const Shape s{B, H, N, d};
+    if (s.n_tiles() > kMaxSelectTiles) return 0;
+    return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + up(select_ws_bytes(s)) + up(mask_bytes(s));
+}
+
+sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
+                                   const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4],
+                                   int B, int H, int N, int d, float sm_scale, float tau, const uint32_t *mask_in,
+                                   uint32_t *mask_out, void *workspace, size_t workspace_bytes, sage_stream_t stream,
+                                   sage_event_t attn_begin, sage_event_t attn_end) {
+    sage_status_t r;
+    if ((r = check_sparse_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
+        (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
+        (r = check_view(out, o_stride, "out")) || (!mask_in && (r = check_tau(tau))) ||
+        (mask_in && (r = check_dev(mask_in, "mask_in", 4))) || (mask_out && (r = check_dev(mask_out, "mask_out", 4))))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    const size_t cb = up(codes_bytes(s)), sb = up(stats_ws_bytes(s)), selb = up(select_ws_bytes(s));
+    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + sb + selb + up(mask_bytes(s)), st))) return r;
+    char *base = static_cast<char *>(scr.ptr);
+    const Codes c = carve_codes(base, s);
+    const StatsWs ws = carve_stats_ws(base + cb, s);
+    const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
+    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, &qs, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    // tau >= 1 keeps every key tile (reading S3): the dense kernel computes the
+    // same result bit for bit without walking step lists
+    const bool dense = !mask_in && tau >= 1.f;
+    const uint32_t *mask = mask_in;
+    if (!mask && (!dense || mask_out)) {
+        uint32_t *m = mask_out ? mask_out : reinterpret_cast<uint32_t *>(base + cb + sb + selb);
+        if ((e = launch_select(s, c.q_i8, c.q_scale, c.k_i8, c.k_scale, sm_scale, tau, base + cb + sb, m, nullptr,
+                               st)) != cudaSuccess)
+            return cuda_fail(e, "block selection");
+        mask = m;
+    } else if (mask_out) {
+        if ((e = cudaMemcpyAsync(mask_out, mask_in, mask_bytes(s), cudaMemcpyDeviceToDevice, st)) != cudaSuccess)
+            return cuda_fail(e, "mask copy");
+    }
+    if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    e = dense ? launch_attention(s, c, dst(out, o_stride), sm_scale, st)
+              : launch_attention_sparse(s, c, dst(out, o_stride), sm_scale, mask, st);
+    if (e != cudaSuccess) return cuda_fail(e, "attention kernel");
+    if (attn_end && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_end), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    return SAGE_OK;
+}
+
 sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4], const void *k,
                                       const int64_t k_stride[4], const void *v, const int64_t v_stride[4], void *out,
                                       const int64_t o_stride[4], int B, int H, int N, int d, float sm_scale,

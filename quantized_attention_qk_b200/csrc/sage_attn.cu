@@ -27,6 +27,13 @@
 // Barriers a waiter tracks by phase parity never get two phases ahead of it:
 // "P ready" has one barrier per P buffer, and the epilogue waits on a barrier
 // committed once after the tile's last PV.
+// Block-sparse instantiation (SPARSE): each Q tile attends only to the key
+// tiles its row of a bit mask selects.  Three warps turn the two mask rows into
+// step lists in shared memory at the start (tile 0's key tiles, tile 1's, and
+// their union with a flag per entry saying which tiles attend), so a step costs
+// one shared load per role.  The producer streams the union through the ring;
+// each tile's QK and PV MMAs, barriers and P buffers advance with the tile's
+// own step count; a tile that keeps no key tile writes zeros.
 // Numerics (readings C4-C8): x = S*(sq*sm_scale*log2e*sk) with one sk per
 // 64-key block; running max m' = max(m, ceil(rowmax x)) so that the O / l
 // rescale 2^(m-m') is an exact power of two; P = e4m3(2^(x-m') * 448) computed as
@@ -80,6 +87,7 @@ struct Ctl {
     uint64_t o_done[2];     // per tile: PV of a step completed
     uint64_t o_final[2];    // per tile: every PV of the tile completed (committed once)
     uint64_t drain;
+    int steps[3];           // SPARSE: own steps of tile 0, of tile 1, union steps
     uint32_t tmem_base;
     AbortState abort;
     float v_scale[D];
@@ -88,8 +96,8 @@ struct Ctl {
 // At least 120 KB so that a second CTA never shares the SM: each CTA takes
 // all 512 tensor-memory columns.  (The tiles need more than that anyway.)
 template <int D>
-constexpr int smem_bytes() {
-    constexpr int need = Cfg<D>::TILE_BYTES + static_cast<int>(sizeof(Ctl<D>)) + 1024;
+constexpr int smem_bytes(int extra = 0) {
+    const int need = Cfg<D>::TILE_BYTES + static_cast<int>(sizeof(Ctl<D>)) + extra + 1024;
     return need > 120 * 1024 ? need : 120 * 1024;
 }
 
@@ -105,7 +113,49 @@ struct AttnParams {
     // debug export of one S tile (EXPORT_S instantiation only)
     int32_t *s_export;
     int bh0, q_tile0, kv_tile0;
+    // SPARSE instantiation: [BH][nqb][mask_words], bit j of row (bh, i) set =
+    // query tile i attends to key tile j
+    const uint32_t *kv_mask;
+    int mask_words;
 };
+
+// Step lists of the SPARSE instantiation, built by one warp from mask rows r0
+// (and r1, may be null) of `words` words, bits at or past n ignored: the
+// indices of the set bits of r0 | r1 in ascending order go to list[], and, if
+// flags is not null, flags[k] = (bit in r0) | (bit in r1) << 1.  Returns the
+// count (every lane).
+__device__ __forceinline__ int build_steps(const uint32_t *r0, const uint32_t *r1, int words, int n, uint16_t *list,
+                                           uint8_t *flags) {
+    const int lane = threadIdx.x & 31;
+    int count = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+        const int w = w0 + lane;
+        uint32_t a = 0u, b = 0u;
+        if (w < words) {
+            const uint32_t keep = (w == words - 1 && (n & 31)) ? (1u << (n & 31)) - 1u : ~0u;
+            a = (r0 ? __ldg(r0 + w) : 0u) & keep;
+            b = (r1 ? __ldg(r1 + w) : 0u) & keep;
+        }
+        uint32_t bits = a | b;
+        const int c = __popc(bits);
+        int incl = c;  // inclusive scan of the lanes' counts
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        int pos = count + incl - c;
+        while (bits) {
+            const int bit = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            list[pos] = static_cast<uint16_t>((w << 5) + bit);
+            if (flags) flags[pos] = static_cast<uint8_t>(((a >> bit) & 1u) | (((b >> bit) & 1u) << 1));
+            ++pos;
+        }
+        count += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    return count;
+}
 
 // 2^k for an integer-valued k <= 0 (exact; 0 below the normal range).
 __device__ __forceinline__ float exp2_int(float k) {
@@ -209,7 +259,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int D, bool EXPORT_S>
+template <int D, bool EXPORT_S, bool SPARSE>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -221,6 +271,10 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     uint8_t *sV = sK + C::STAGES * C::K_BYTES;
     uint8_t *sP = sV + C::STAGES * C::V_BYTES;  // [tile][buffer] P tiles
     Ctl<D> *ctl = reinterpret_cast<Ctl<D> *>(sP + 4 * C::P_BYTES);
+    // SPARSE step lists: tile 0's and tile 1's key tiles, the union, its flags
+    uint16_t *slist = reinterpret_cast<uint16_t *>(ctl + 1);
+    uint16_t *ulist = slist + 2 * (SPARSE ? p.nqb : 0);
+    uint8_t *uflag = reinterpret_cast<uint8_t *>(ulist + (SPARSE ? p.nqb : 0));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int bh = EXPORT_S ? p.bh0 : static_cast<int>(blockIdx.y);
@@ -252,6 +306,17 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         if (!EXPORT_S) tma_prefetch_desc(&tm_v);
     }
     for (int i = threadIdx.x; i < D; i += blockDim.x) ctl->v_scale[i] = EXPORT_S ? 0.f : p.v_scale[bh * D + i];
+    if constexpr (SPARSE) {
+        // a tile past the last query tile keeps nothing
+        if (warp < 3) {
+            const uint32_t *r0 = p.kv_mask + ((size_t)bh * p.nqb + qt0) * p.mask_words;
+            const uint32_t *r1 = qt0 + 1 < p.nqb ? r0 + p.mask_words : nullptr;
+            const int n = warp < 2 ? build_steps(warp == 0 ? r0 : r1, nullptr, p.mask_words, nkv,
+                                                 slist + warp * p.nqb, nullptr)
+                                   : build_steps(r0, r1, p.mask_words, nkv, ulist, uflag);
+            if (lane == 0) ctl->steps[warp] = n;
+        }
+    }
     if (warp == 9) {
         tmem_alloc(&ctl->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
@@ -269,15 +334,17 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, qt0 * C::BM, bh);
             tma_load_3d(sQ + C::Q_BYTES, &tm_q, &ctl->q_full, 0, (qt0 + 1) * C::BM, bh);
             int issued = 0;
-            for (int j = 0; j < nkv; ++j) {
+            const int nsteps = SPARSE ? ctl->steps[2] : nkv;
+            for (int j = 0; j < nsteps; ++j) {
+                const int kt = SPARSE ? ulist[j] : j;  // key tile of step j
                 const int s = j % C::STAGES;
                 if (j >= C::STAGES &&
                     !wait_one(&ctl->kv_empty[s], ((j / C::STAGES) - 1) & 1, p.err, &ctl->abort, false, 1))
                     break;
                 mbar_arrive_expect_tx(&ctl->kv_full[s], EXPORT_S ? C::K_BYTES : C::K_BYTES + C::V_BYTES);
-                tma_load_3d(sK + s * C::K_BYTES, &tm_k, &ctl->kv_full[s], 0, (kv0 + j) * C::BN, bh);
+                tma_load_3d(sK + s * C::K_BYTES, &tm_k, &ctl->kv_full[s], 0, (kv0 + kt) * C::BN, bh);
                 if (!EXPORT_S)
-                    tma_load_3d(sV + s * C::V_BYTES, &tm_v, &ctl->kv_full[s], 0, (kv0 + j) * C::BN, bh);
+                    tma_load_3d(sV + s * C::V_BYTES, &tm_v, &ctl->kv_full[s], 0, (kv0 + kt) * C::BN, bh);
                 issued = j + 1;
             }
             // every copy started here lands before the CTA may exit
@@ -307,16 +374,70 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 mma_i8_ss_if(me, tmem + t * 128, a + 2 * kk, b + 2 * kk, idesc_qk, kk > 0 ? 1u : 0u);
             tc_commit_if(me, &ctl->s_full[t]);
         };
-        auto issue_pv = [&](int t, int s, int j) {
-            const uint64_t a = dp + (uint64_t)((((2 * t + (j & 1)) * C::P_BYTES)) >> 4);
+        // n: the tile's own step (P buffer n % 2; O accumulates after its first)
+        auto issue_pv = [&](int t, int s, int n, bool last) {
+            const uint64_t a = dp + (uint64_t)((((2 * t + (n & 1)) * C::P_BYTES)) >> 4);
             const uint64_t b = dv + (uint64_t)((s * C::V_BYTES) >> 4);
 #pragma unroll
             for (int kk = 0; kk < C::BN / 32; ++kk)
                 mma_f8_ss_if(me, tmem + C::T_O + t * D, a + 2 * kk, b + 2 * kk * D, idesc_pv,
-                             (j > 0 || kk > 0) ? 1u : 0u);
+                             (n > 0 || kk > 0) ? 1u : 0u);
             tc_commit_if(me, &ctl->o_done[t]);
-            if (j == nkv - 1) tc_commit_if(me, &ctl->o_final[t]);
+            if (last) tc_commit_if(me, &ctl->o_final[t]);
         };
+        if constexpr (SPARSE) {
+            // union step u streams key tile kt; tile t runs its own steps
+            // PVs go in union order; each tile's next QK goes out as soon as its
+            // K tile is in the ring (within STAGES-1 union steps), its S buffer
+            // is free and PV(n-2) of that tile is issued (so S(n) finishing still
+            // proves P buffer n%2 free).  With every tile kept this is the dense
+            // issue order.
+            const int tot[2] = {ctl->steps[0], ctl->steps[1]}, nu = ctl->steps[2];
+            int nq[2] = {0, 0}, np[2] = {0, 0};  // QK and PV MMAs issued per tile
+            int cq[2];                           // union step of each tile's next QK
+            auto next_of = [&](int t, int from) {
+                while (from < nu && !((uflag[from] >> t) & 1u)) ++from;
+                return from;
+            };
+            cq[0] = next_of(0, 0);
+            cq[1] = next_of(1, 0);
+            bool ok = wait_warp(&ctl->q_full, 0, p.err, &ctl->abort, 4);
+            for (int t = 0; ok && t < 2; ++t) {
+                const int v = cq[t];
+                if (v >= nu || v > C::STAGES - 1) continue;
+                if (!(ok = wait_warp(&ctl->kv_full[v % C::STAGES], (v / C::STAGES) & 1, p.err, &ctl->abort, 5)))
+                    break;
+                tc_fence_after();
+                issue_qk(t, v % C::STAGES);
+                nq[t] = 1;
+                cq[t] = next_of(t, v + 1);
+            }
+            for (int u = 0; ok && u < nu; ++u) {
+                const int s = u % C::STAGES;
+                for (int t = 0; ok && t < 2; ++t) {
+                    const int v = cq[t], n = nq[t];
+                    if (v >= nu || v > u + C::STAGES - 1 || np[t] < n - 1) continue;
+                    if (!(ok = wait_warp(&ctl->kv_full[v % C::STAGES], (v / C::STAGES) & 1, p.err, &ctl->abort, 6)))
+                        break;
+                    // the tile's softmax holds its previous S in registers already
+                    if (n > 0 && !(ok = wait_warp(&ctl->s_free[t], (n - 1) & 1, p.err, &ctl->abort, 7))) break;
+                    tc_fence_after();
+                    issue_qk(t, v % C::STAGES);
+                    nq[t] = n + 1;
+                    cq[t] = next_of(t, v + 1);
+                }
+                const uint32_t fl = uflag[u];  // tiles attending union step u
+                for (int t = 0; ok && t < 2; ++t) {
+                    if (!((fl >> t) & 1u)) continue;
+                    const int n = np[t];
+                    if (!(ok = wait_warp(&ctl->p_ready[t][n & 1], (n >> 1) & 1, p.err, &ctl->abort, 8))) break;
+                    tc_fence_after();
+                    issue_pv(t, s, n, n == tot[t] - 1);
+                    np[t] = n + 1;
+                }
+                if (ok) tc_commit_if(me, &ctl->kv_empty[s]);
+            }
+        } else {
         bool ok = wait_warp(&ctl->q_full, 0, p.err, &ctl->abort, 4) &&
                   wait_warp(&ctl->kv_full[0], 0, p.err, &ctl->abort, 5);
         if (ok) {
@@ -340,9 +461,10 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             for (int t = 0; ok && t < 2; ++t) {
                 if (!(ok = wait_warp(&ctl->p_ready[t][j & 1], (j >> 1) & 1, p.err, &ctl->abort, 8))) break;
                 tc_fence_after();
-                if (!EXPORT_S) issue_pv(t, s, j);
+                if (!EXPORT_S) issue_pv(t, s, j, j == nkv - 1);
             }
             if (ok) tc_commit_if(me, &ctl->kv_empty[s]);
+        }
         }
         // all MMAs issued here finish before tensor memory is released
         tc_commit_if(me, &ctl->drain);
@@ -364,15 +486,21 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         const float cq = sq * p.s_l2;
         const float kLog2_448 = 8.807354922057604f;
         const float *ksc = p.k_scale + (int64_t)bh * p.nkb + 2 * kv0;
+        const uint16_t *mylist = slist + t * (SPARSE ? p.nqb : 0);
+        const int steps = SPARSE ? ctl->steps[t] : nkv;  // this tile's own steps
+        int kt_next = (SPARSE && steps > 0) ? mylist[0] : 0;  // key tile of the next step
         float m = -INFINITY, l = 0.f;
-        float ks_next0 = EXPORT_S ? 0.f : __ldg(ksc), ks_next1 = EXPORT_S ? 0.f : __ldg(ksc + 1);
+        float ks_next0 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next);
+        float ks_next1 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next + 1);
         bool ok = true;
-        for (int j = 0; ok && j < nkv; ++j) {
-            // this step's two K-block scales were fetched one step ahead
+        for (int j = 0; ok && j < steps; ++j) {
+            // this step's key tile and its two K-block scales were fetched one step ahead
+            const int kt = kt_next;
             const float ks0 = ks_next0, ks1 = ks_next1;
-            if (!EXPORT_S && j + 1 < nkv) {
-                ks_next0 = __ldg(ksc + 2 * (j + 1));
-                ks_next1 = __ldg(ksc + 2 * (j + 1) + 1);
+            if (!EXPORT_S && j + 1 < steps) {
+                kt_next = SPARSE ? mylist[j + 1] : j + 1;
+                ks_next0 = __ldg(ksc + 2 * kt_next);
+                ks_next1 = __ldg(ksc + 2 * kt_next + 1);
             }
             if (!(ok = wait_warp(&ctl->s_full[t], j & 1, p.err, &ctl->abort, 10 + t))) break;
             tc_fence_after();
@@ -401,7 +529,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     }
                 }
             } else {
-                const int n_valid = min(C::BN, p.N - (kv0 + j) * C::BN);
+                const int n_valid = min(C::BN, p.N - (kv0 + kt) * C::BN);
                 const float c0 = cq * ks0, c1 = cq * ks1;
                 float x0, x1;
                 if (n_valid == C::BN) {
@@ -484,7 +612,15 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&ctl->p_ready[t][j & 1]);
         }
-        if (ok && !EXPORT_S && wait_warp(&ctl->o_final[t], 0, p.err, &ctl->abort, 13)) {
+        if (SPARSE && steps == 0) {
+            // the tile keeps no key tile: its rows have no softmax and are 0
+            if (grow < p.N) {
+                uint4 *dst = reinterpret_cast<uint4 *>(p.out + (int64_t)(bh / p.H) * p.osb +
+                                                       (int64_t)(bh % p.H) * p.osh + (int64_t)grow * p.osn);
+#pragma unroll
+                for (int i = 0; i < D / 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        } else if (ok && !EXPORT_S && wait_warp(&ctl->o_final[t], 0, p.err, &ctl->abort, 13)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
             uint16_t *orow = p.out + (int64_t)(bh / p.H) * p.osb + (int64_t)(bh % p.H) * p.osh +
@@ -554,7 +690,7 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
 }
 
 
-template <int D, bool EXPORT_S>
+template <int D, bool EXPORT_S, bool SPARSE>
 cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
                           const AttnParams &p0, dim3 grid, cudaStream_t st) {
     using C = Cfg<D>;
@@ -571,8 +707,9 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     AttnParams p = p0;
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorSymbolNotFound;
-    const int smem = smem_bytes<D>();
-    auto kern = k_attn<D, EXPORT_S>;
+    const int smem = smem_bytes<D>(SPARSE ? 7 * p.nqb + 8 : 0);  // three uint16 lists and one uint8 list
+    if (smem > 227 * 1024) return cudaErrorInvalidValue;
+    auto kern = k_attn<D, EXPORT_S, SPARSE>;
     // The setmaxnreg split assumes the kernel is launched with LAUNCH_REGS per
     // thread; with fewer the increases could never be satisfied.
     cudaFuncAttributes fa;
@@ -642,8 +779,30 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
     p.nkb = s.n_kblocks();
     p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
-    return s.d == 128 ? launch_attn_d<128, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
-                      : launch_attn_d<64, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
+    return s.d == 128 ? launch_attn_d<128, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
+                      : launch_attn_d<64, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
+}
+
+cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,
+                                    const uint32_t *kv_mask, cudaStream_t st) {
+    AttnParams p{};
+    p.q_scale = c.q_scale;
+    p.k_scale = c.k_scale;
+    p.v_scale = c.v_scale;
+    p.out = out.p;
+    p.osb = out.sb;
+    p.osh = out.sh;
+    p.osn = out.sn;
+    p.H = s.H;
+    p.N = s.N;
+    p.nqb = s.n_qblocks();
+    p.nkb = s.n_kblocks();
+    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    p.kv_mask = kv_mask;
+    p.mask_words = s.mask_words();
+    dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
+    return s.d == 128 ? launch_attn_d<128, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
+                      : launch_attn_d<64, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
 }
 
 cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,
@@ -657,8 +816,8 @@ cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_
     p.bh0 = bh;
     p.q_tile0 = q_tile;
     p.kv_tile0 = kv_tile;
-    return s.d == 128 ? launch_attn_d<128, true>(s, q_i8, k_i8, nullptr, p, dim3(1, 1), st)
-                      : launch_attn_d<64, true>(s, q_i8, k_i8, nullptr, p, dim3(1, 1), st);
+    return s.d == 128 ? launch_attn_d<128, true, false>(s, q_i8, k_i8, nullptr, p, dim3(1, 1), st)
+                      : launch_attn_d<64, true, false>(s, q_i8, k_i8, nullptr, p, dim3(1, 1), st);
 }
 
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st) {

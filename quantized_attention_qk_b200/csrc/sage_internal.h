@@ -14,6 +14,7 @@ constexpr int kKBlock = 64;        // K tokens per quantization block
 constexpr int kKvTile = 128;       // keys per attention KV tile (two K blocks)
 constexpr int kStatsRows = 256;    // statistics pass: tokens per chunk (a multiple of 64)
 constexpr unsigned kErrTimeoutBit = 1u;  // device error word: a bounded wait gave up
+constexpr int kMaxSelectTiles = 4096;    // block-sparse selection: key tiles one row ranks in shared memory
 
 // A bf16 [B,H,N,d] tensor given by base pointer and element strides (c stride 1).
 struct Src {
@@ -37,6 +38,10 @@ struct Shape {
     // share the call.
     int chunk_rows() const { return kStatsRows; }
     int n_chunks() const { return (N + chunk_rows() - 1) / chunk_rows(); }
+    // Block-sparse masks: one row of mask_words() 32-bit words per (b,h, query
+    // tile), bit j = key tile j (tiles of kKvTile tokens for both).
+    int n_tiles() const { return (N + kKvTile - 1) / kKvTile; }
+    int mask_words() const { return (n_tiles() + 31) / 32; }
 };
 
 // Scratch of the quantize pass: per-chunk partials and the finished statistics.
@@ -80,9 +85,19 @@ unsigned *device_error_ptr();
 
 // Attention launchers (sage_attn.cu).
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);
+cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,
+                                    const uint32_t *kv_mask, cudaStream_t st);
 cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,
                                  int kv_tile, int32_t *s_out, cudaStream_t st);
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st);
+
+// Block-sparse selection (sage_sparse.cu): scratch for the pooled tile
+// vectors, the mask size, and the launcher (scores, ranking, kept prefix).
+size_t select_ws_bytes(const Shape &s);
+size_t mask_bytes(const Shape &s);
+cudaError_t launch_select(const Shape &s, const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                          const float *k_scale, float sm_scale, float tau, void *ws, uint32_t *mask, float *sbar_out,
+                          cudaStream_t st);
 
 // Dense fp32 reference (sage_dense_ref.cu).
 cudaError_t launch_dense_ref(const Shape &s, const Src &q, const Src &k, const Src &v, const Dst &out,

@@ -102,3 +102,58 @@ def test_host_forward_rejects_bad_arguments_before_any_launch(L):
     L.sage_attn_fwd_host_scratch_bytes.restype = ctypes.c_size_t
     assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 128) > 3 * 24 * 4608 * 128 * 2 + 24 * 4608 * 128 * 2
     assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 96) == 0
+
+
+def _call_sparse(L, tau=0.5, N=128, d=64, mask_in=None, mask_out=None, q=16 * 4096):
+    st = (ctypes.c_int64 * 4)(8 * 4096, 4096 * 8, 8 * 8, 1)
+    p = ctypes.c_void_p(q)
+    return L.sage_attn_fwd_sparse(p, st, p, st, p, st, p, st, 1, 1, N, d, ctypes.c_float(0.125), ctypes.c_float(tau),
+                                  mask_in, mask_out, None, 0, None, None, None)
+
+
+def test_sparse_sizes_and_schedule(L):
+    # one mask row of ceil(T/32) words per (b,h, query tile)
+    for (B, H, N) in [(1, 2, 256), (1, 24, 4608), (1, 40, 34020), (2, 3, 4097)]:
+        T = -(-N // 128)
+        assert sage.sage_block_mask_bytes(B, H, N) == B * H * T * (-(-T // 32)) * 4
+        assert sage.sage_attn_sparse_workspace_bytes(B, H, N, 128) > sage.sage_attn_workspace_bytes(B, H, N, 128)
+    assert sage.sage_block_mask_bytes(1, 1, 4096 * 128) > 0
+    assert sage.sage_block_mask_bytes(1, 1, 4096 * 128 + 1) == 0
+    assert sage.sage_attn_sparse_workspace_bytes(1, 1, 128, 96) == 0
+    assert sage.sage_tau_schedule(0, 11, 0.5, 1.0) == 0.5
+    assert sage.sage_tau_schedule(10, 11, 0.5, 1.0) == 1.0
+    assert sage.sage_tau_schedule(5, 11, 0.5, 1.0) == pytest.approx(0.75, abs=1e-7)
+    assert sage.sage_tau_schedule(-4, 11, 0.5, 1.0) == 0.5
+    assert sage.sage_tau_schedule(40, 11, 0.5, 1.0) == 1.0
+    assert sage.sage_tau_schedule(3, 1, 0.2, 0.9) == pytest.approx(0.9)
+
+
+def test_sparse_calls_reject_bad_arguments_before_any_launch(L):
+    for tau in (0.0, -1.0, float("nan"), float("inf")):
+        assert _call_sparse(L, tau=tau) == 1, tau
+        assert "tau" in L.sage_last_error_message().decode()
+    assert _call_sparse(L, N=4096 * 128 + 1) == 2                       # too many tiles
+    assert _call_sparse(L, mask_in=ctypes.c_void_p(4 * 4096 + 2)) == 1  # misaligned mask
+    assert _call_sparse(L, mask_out=ctypes.c_void_p(4 * 4096 + 1)) == 1
+    assert _call_sparse(L, d=96) == 2
+    st = ctypes.c_void_p(16 * 4096)
+    assert L.sage_block_select(st, st, st, st, 1, 1, 256, 64, ctypes.c_float(0.125), ctypes.c_float(0.0), st, None,
+                               None, 0, None) == 1
+    assert L.sage_block_select(st, st, st, st, 1, 1, 256, 64, ctypes.c_float(0.125), ctypes.c_float(0.5), None, None,
+                               None, 0, None) == 1                      # null mask
+    import torch
+    with pytest.raises(ValueError):  # host tensors: refused, never computed elsewhere
+        sage.sage_attn_fwd_sparse(*(torch.zeros(1, 1, 128, 64, dtype=torch.bfloat16) for _ in range(3)), tau=0.5)
+
+
+def test_mask_packing_round_trips():
+    import torch
+    g = torch.Generator().manual_seed(3)
+    for T in (1, 31, 32, 33, 70):
+        keep = torch.rand(2, 1, T, T, generator=g) < 0.4
+        m = sage.keep_to_mask(keep)
+        assert m.shape == (2, 1, T, -(-T // 32)) and m.dtype == torch.int32
+        assert torch.equal(sage.mask_to_keep(m, T), keep)
+        # bit j of word j // 32
+        j = T - 1
+        assert bool(((m[0, 0, 0, j // 32].item() & 0xFFFFFFFF) >> (j % 32)) & 1) == bool(keep[0, 0, 0, j])

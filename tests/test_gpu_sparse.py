@@ -1,0 +1,213 @@
+"""GPU parity of block-sparse skipping (readings S1-S4 of the sol-attn page's
+scheduled sparsity) through the C ABI.
+
+* every key tile kept (tau = 1, or an all-ones mask): bit for bit the dense
+  forward;
+* a mask the test draws (seeded; rows that keep nothing, only the ragged tail
+  tile, everything; the two query tiles of a CTA with disjoint masks): the
+  output against the oracle's masked quant emulation with that same mask,
+  within the scheme's tolerances (relative L2 <= 2e-3, max |diff| <= 1e-2);
+* the GPU's tile scores against the oracle's (each side from its own codes)
+  and the GPU's kept sets against the properties that define reading S3,
+  with the oracle's mass; where the two rankings agree at the cut the kept
+  sets are equal;
+* the full flux workload with a drawn mask on sampled heads and rows.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_qk_b200 as sage
+from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv, tiny_custom
+from tests import _gpu_util as U
+
+pytestmark = [pytest.mark.gpu, pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")]
+
+DEV = "cuda"
+T = 128
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from quantized_attention_qk_b200 import build
+    build.build()
+    oracle.build()
+
+
+def _inputs(w, planted=False):
+    q, k, v, _ = make_qkv(w)
+    if planted:
+        q, k = _plant(q, k, w.seed)
+    return (q, k, v), tuple(t.to(DEV) for t in (q, k, v))
+
+
+def _plant(q, k, seed):
+    """Give each query / key tile its own offset vector so that tile scores
+    differ (iid inputs make every tile pair look alike)."""
+    B, H, N, d = q.shape
+    nt = -(-N // T)
+    g = torch.Generator().manual_seed(seed + 99)
+    uq = torch.randn(B, H, nt, d, generator=g) * 0.6
+    uk = torch.randn(B, H, nt, d, generator=g) * 0.6
+    q = q.float() + uq.repeat_interleave(T, dim=2)[:, :, :N]
+    k = k.float() + uk.repeat_interleave(T, dim=2)[:, :, :N]
+    return q.to(torch.bfloat16), k.to(torch.bfloat16)
+
+
+def _draw_keep(B, H, N, seed, density=0.5):
+    nt = -(-N // T)
+    rng = np.random.default_rng(seed)
+    keep = (rng.random((B, H, nt, nt)) < density).astype(np.uint8)
+    keep[..., 0, :] = 0                       # a query tile that keeps nothing
+    if nt > 1:
+        keep[..., 1, :] = 0
+        keep[..., 1, nt - 1] = 1              # one that keeps only the ragged tail tile
+    if nt > 2:
+        keep[..., 2, :] = 1                   # one that keeps everything
+    if nt > 4:                                # CTA of tiles 4, 5: disjoint rows
+        keep[..., 4, :] = 0
+        keep[..., 4, ::2] = 1
+        keep[..., 5, :] = 0
+        keep[..., 5, 1::2] = 1
+    return keep
+
+
+def _run_masked(dev_qkv, w, keep):
+    mask = sage.keep_to_mask(torch.from_numpy(keep).to(DEV))
+    out, used = sage.sage_attn_fwd_sparse(*dev_qkv, sm_scale=w.sm_scale, mask=mask, return_mask=True)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(used, mask)
+    return out
+
+
+@pytest.mark.parametrize("w", [
+    tiny_custom(1, 2, 300, 64, 501, bias_sigma=2.0),
+    tiny_custom(2, 1, 520, 128, 502, layout="fused", bias_sigma=4.0, outlier_frac=0.01),
+    WORKLOADS["tiny"],
+], ids=lambda w: w.name)
+def test_every_tile_kept_is_the_dense_forward_bit_for_bit(w):
+    _, dev = _inputs(w)
+    dense = sage.sage_attn_fwd(*dev, sm_scale=w.sm_scale)
+    sp = sage.sage_attn_fwd_sparse(*dev, tau=1.0, sm_scale=w.sm_scale)
+    nt = -(-w.N // T)
+    ones = _run_masked(dev, w, np.ones((w.B, w.H, nt, nt), np.uint8))
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(sp, dense)
+    assert torch.equal(ones, dense)
+
+
+@pytest.mark.parametrize("w,density", [
+    (tiny_custom(1, 2, 300, 64, 511, bias_sigma=2.0), 0.5),
+    (tiny_custom(1, 2, 777, 128, 512, layout="fused", bias_sigma=4.0, outlier_frac=0.01), 0.4),
+    (tiny_custom(2, 1, 1280, 64, 513, bias_sigma=2.0), 0.25),
+    (tiny_custom(1, 1, 129, 128, 514), 0.5),
+], ids=lambda x: getattr(x, "name", str(x)))
+def test_drawn_mask_matches_the_masked_oracle(w, density):
+    (q, k, v), dev = _inputs(w)
+    keep = _draw_keep(w.B, w.H, w.N, w.seed, density)
+    out = _run_masked(dev, w, keep)
+    got = U.bf16_to_f64(out)
+    _, bits = oracle.attn_quant(q, k, v, w.sm_scale, kv_keep=keep)
+    want = oracle.bf16_bits_to_f64(bits)
+    ok, rel, mx = U.within_tol(got, want)
+    assert np.isfinite(got).all()
+    assert ok, (w.name, rel, mx)
+    assert np.all(got[:, :, :T] == 0.0)       # tile 0 keeps nothing
+
+
+def _check_selection(keep_gpu, sbar_o, N, tau):
+    """GPU kept sets against reading S3 with the oracle's scores and fp64 mass.
+    Returns the fraction of rows whose kept set equals the oracle's."""
+    nt = sbar_o.shape[-1]
+    n = np.array([min(T, N - j * T) for j in range(nt)], dtype=np.float64)
+    keep_o = oracle.block_select(sbar_o, N, tau)
+    same = 0
+    rows = 0
+    for idx in np.ndindex(*sbar_o.shape[:-1]):
+        rows += 1
+        kg, ko = keep_gpu[idx].astype(bool), keep_o[idx].astype(bool)
+        if np.array_equal(kg, ko):
+            same += 1
+            continue
+        row = sbar_o[idx].astype(np.float64)
+        w = n * np.exp2(row - row.max())
+        tot = w.sum()
+        assert kg.sum() >= 1
+        # the GPU may cut one tile earlier or later only where the oracle's
+        # mass sits at tau within fp32 accumulation error, and may order only
+        # near-equal scores differently
+        kept_min = row[kg].min()
+        dropped_max = row[~kg].max() if (~kg).any() else -np.inf
+        assert dropped_max <= kept_min + 1e-4 * max(1.0, abs(kept_min)), idx
+        mass = w[kg].sum()
+        assert mass >= tau * tot * (1 - 1e-4), (idx, mass / tot, tau)
+        assert mass - w[kg][np.argmin(row[kg])] < tau * tot * (1 + 1e-4), (idx, mass / tot, tau)
+    return same / rows
+
+
+@pytest.mark.parametrize("w", [
+    tiny_custom(1, 3, 1500, 128, 521, bias_sigma=4.0, outlier_frac=0.01),
+    tiny_custom(2, 2, 2100, 64, 522, bias_sigma=2.0),
+], ids=lambda w: w.name)
+def test_selection_matches_the_oracle(w):
+    (q, k, v), dev = _inputs(w, planted=True)
+    codes = sage.sage_quant_qk(dev[0], dev[1])
+    sbar_o = oracle.block_scores(q, k, v, w.sm_scale)
+    for tau in (0.3, 0.6, 0.9, 0.999):
+        mask, sbar_g = sage.sage_block_select(codes, w.N, w.sm_scale, tau, want_scores=True)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        sg = sbar_g.cpu().numpy()
+        scale = np.abs(sbar_o).max()
+        assert np.max(np.abs(sg - sbar_o)) <= 2e-3 * scale, tau
+        keep_g = sage.mask_to_keep(mask, sbar_o.shape[-1]).cpu().numpy()
+        frac_same = _check_selection(keep_g, sbar_o, w.N, tau)
+        assert frac_same >= 0.97, (tau, frac_same)
+    # the forward's own selection is the same mask
+    out, used = sage.sage_attn_fwd_sparse(*dev, tau=0.6, sm_scale=w.sm_scale, return_mask=True)
+    again = sage.sage_block_select(codes, w.N, w.sm_scale, 0.6)
+    torch.cuda.synchronize()
+    assert torch.equal(used, again)
+
+
+def test_tau_forward_matches_the_oracle_where_the_masks_agree():
+    w = tiny_custom(1, 2, 1100, 128, 531, bias_sigma=4.0)
+    (q, k, v), dev = _inputs(w, planted=True)
+    out, mask = sage.sage_attn_fwd_sparse(*dev, tau=0.5, sm_scale=w.sm_scale, return_mask=True)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    nt = -(-w.N // T)
+    keep_g = sage.mask_to_keep(mask, nt).cpu().numpy()
+    keep_o = oracle.block_select(oracle.block_scores(q, k, v, w.sm_scale), w.N, 0.5)
+    agree = np.all(keep_g == keep_o, axis=-1)           # [B,H,nt] rows with the same kept set
+    assert agree.mean() >= 0.9
+    assert keep_o.sum() < 0.8 * keep_o.size              # the selection really skips tiles
+    _, bits = oracle.attn_quant(q, k, v, w.sm_scale, kv_keep=keep_o)
+    want = oracle.bf16_bits_to_f64(bits)
+    got = U.bf16_to_f64(out)
+    for b in range(w.B):
+        for h in range(w.H):
+            for i in np.nonzero(agree[b, h])[0]:
+                sl = slice(i * T, min(w.N, (i + 1) * T))
+                ok, rel, mx = U.within_tol(got[b, h, sl], want[b, h, sl])
+                assert ok, (b, h, i, rel, mx)
+
+
+def test_flux_workload_with_a_drawn_mask_on_sampled_rows():
+    w = WORKLOADS["flux"]
+    (q, k, v), dev = _inputs(w)
+    keep = _draw_keep(w.B, w.H, w.N, 541, density=0.5)
+    out = _run_masked(dev, w, keep)
+    heads = [(0, 0), (0, 13), (0, 23)]
+    rows = U.sample_rows(w.N, 48, 7)
+    got = U.stack(U.gather(out, heads, rows), heads)
+    want = []
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        _, bits = oracle.attn_quant(q[sl], k[sl], v[sl], w.sm_scale, rows=rows, kv_keep=keep[sl])
+        want.append(oracle.bf16_bits_to_f64(bits[0, 0]))
+    ok, rel, mx = U.within_tol(got, np.stack(want))
+    assert ok, (rel, mx)
