@@ -211,3 +211,18 @@ def test_flux_workload_with_a_drawn_mask_on_sampled_rows():
         want.append(oracle.bf16_bits_to_f64(bits[0, 0]))
     ok, rel, mx = U.within_tol(got, np.stack(want))
     assert ok, (rel, mx)
+
+
+def test_single_tile_sequences():
+    w = tiny_custom(1, 2, 77, 64, 551, layout="fused", bias_sigma=2.0)
+    _, dev = _inputs(w)
+    dense = sage.sage_attn_fwd(*dev, sm_scale=w.sm_scale)
+    full = _run_masked(dev, w, np.ones((1, 2, 1, 1), np.uint8))
+    empty = _run_masked(dev, w, np.zeros((1, 2, 1, 1), np.uint8))
+    sel, mask = sage.sage_attn_fwd_sparse(*dev, tau=0.2, sm_scale=w.sm_scale, return_mask=True)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(full, dense)
+    assert torch.count_nonzero(empty).item() == 0
+    assert torch.equal(sel, dense)  # one tile: every tau keeps it
+    assert sage.mask_to_keep(mask, 1).all()
