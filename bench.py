@@ -196,14 +196,18 @@ def run_gpu(args):
         q, k, v, bufs = make_qkv(w, device=dev)
         out = torch.empty(w.B, w.H, w.N, w.d, dtype=torch.bfloat16, device=dev)
         sparse = args.tau is not None
-        ws_bytes = (sage.sage_attn_sparse_workspace_bytes if sparse else sage.sage_attn_workspace_bytes)(
-            w.B, w.H, w.N, w.d)
+        ws_fn = (sage.sage_attn_sparse_workspace_bytes if sparse else
+                 sage.sage_attn_kres_workspace_bytes if args.kres else sage.sage_attn_workspace_bytes)
+        ws_bytes = ws_fn(w.B, w.H, w.N, w.d)
         ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
 
         def forward(events=None):
             if sparse:
                 return sage.sage_attn_fwd_sparse(q, k, v, tau=args.tau, sm_scale=w.sm_scale, out=out, workspace=ws,
                                                  attn_events=events)
+            if args.kres:
+                return sage.sage_attn_fwd_kres(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws,
+                                               attn_events=events)
             return sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws, attn_events=events)
 
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -278,14 +282,15 @@ def run_gpu(args):
                    "l2": "flushed before every timed step (256 MB write, outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "k_attn (fused attention)", "achieved": round(attn_tops, 2),
                      "peak": round(peak_8bit, 1), "unit": "TFLOP/s", "frac": round(attn_tops / peak_8bit, 4),
-                     "traffic": None if args.tau is not None else _attn_traffic(wp.name),
+                     "traffic": None if (args.tau is not None or args.kres) else _attn_traffic(wp.name),
                      "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
                        "attention, bf16 out -> pinned host; dense)"},
-        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.tau is not None and args.tau < 1 else 0)) * args.steps,
+        "gpu_launches": (LAUNCHES_PER_STEP + (3 if args.tau is not None and args.tau < 1 else 0) +
+                         (2 if args.kres else 0)) * args.steps,
         "clocks": r["clocks"],
     }
     if args.tau is not None:
@@ -293,7 +298,10 @@ def run_gpu(args):
         line["config"]["kept_fraction"] = round(r["kept"], 4)
         line["config"]["ops"] = ("value counts the dense 4*B*H*N^2*d; roofline.achieved counts the kept tile "
                                  "pairs only (block-sparse forward, sage_attn_fwd_sparse)")
-    if args.secondary and args.workload != SECONDARY and args.tau is None:
+    if args.kres:
+        line["config"]["k_residual"] = ("K-residual quantization (sage_attn_fwd_kres): residual codes per 64-token "
+                                        "block, bf16 block means, mean term on the tensor cores")
+    if args.secondary and args.workload != SECONDARY and args.tau is None and not args.kres:
         ws_ = WORKLOADS[SECONDARY]
         r2 = measure(ws_, max(3, args.steps // 2), args.warmup)
         k2 = max(3, args.steps // 2)
@@ -354,6 +362,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--tau", type=float, default=None,
                     help="time the block-sparse forward with this tau instead of the dense one")
+    ap.add_argument("--kres", action="store_true",
+                    help="time the K-residual forward instead of the smoothing one")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

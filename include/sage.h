@@ -21,7 +21,8 @@
  *          the dense formula with the 1/sqrt(d_k) scale (the dense reference).
  *   [BLOG] "GitHub榜单静默期：Attention优化从架构转向推理加速", section 2.2:
  *          block-wise computation that never writes the attention matrix out.
- *   [SOL]  "ComfyUI-sol-attn" page, "核心亮点" items 2 and 4: zero-copy reads of a
+ *   [SOL]  "ComfyUI-sol-attn" page, "核心亮点" items 1, 2 and 4: K-residual
+ *          quantization with the block-mean term kept at bf16; zero-copy reads of a
  *          fused-qkv strided view; explicit, logged rejection of unsupported
  *          inputs instead of a silent fallback; scheduled sparsity, a value
  *          tau that may ramp over the sampling steps (sparse early, dense late).
@@ -304,6 +305,49 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4],
  * from sparse (small tau) early to dense (tau = 1) late.  Host function.
  */
 float sage_tau_schedule(int step, int n_steps, float tau_start, float tau_end);
+
+/* ------------------------------------------------------------------------ */
+/* K-residual quantization ([SOL] item 1: quantize only the residual of K     */
+/* inside each block; keep the block-mean term at bf16 precision).  Readings  */
+/* where the page is silent: the blocks are the 64-token K blocks; the block  */
+/* mean is the mean of the block's valid tokens (summed exactly), rounded to  */
+/* bf16; the residual fp32(k) - fp32(mean) is coded as the other INT8 codes;  */
+/* every score of row r against a key of block b gains                        */
+/* e[r][b] = (q_r . mean_b) * fp32(sm_scale * log2 e), from the bf16 inputs   */
+/* with fp32 accumulation.  No smoothing by the global mean in this mode.     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * sage_quant_k_residual -- the residual codes of K: k_i8 [B,H,N_pad,d] int8
+ * (padded rows 0), k_scale [B,H,N_pad/64] fp32, k_bmean [B,H,N_pad/64,d] bf16
+ * bit patterns (blocks past N: 0), all device buffers (k_bmean 16-byte aligned).
+ */
+sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4],
+                                    int B, int H, int N, int d,
+                                    int8_t *k_i8, float *k_scale, uint16_t *k_bmean,
+                                    sage_stream_t stream);
+
+/* Bytes of scratch sage_attn_fwd_kres needs (0 for a shape rejected): the
+ * codes, the V statistics, the bf16 block means and the fp32 mean term
+ * ([B*H][N_pad/64][N_pad], 4*B*H*N_pad^2/64 bytes). */
+size_t sage_attn_kres_workspace_bytes(int B, int H, int N, int d);
+
+/*
+ * sage_attn_fwd_kres -- the forward with K-residual quantization instead of
+ * the smoothing: Q and V coded as in sage_attn_fwd, K as in
+ * sage_quant_k_residual, the mean term computed on the tensor cores (bf16
+ * products, fp32 accumulation), and the fused attention kernel adding it to
+ * each score's exponent.  Arguments, layouts, events and errors as
+ * sage_attn_fwd_ev.
+ */
+sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4],
+                                 const void *k, const int64_t k_stride[4],
+                                 const void *v, const int64_t v_stride[4],
+                                 void *out, const int64_t o_stride[4],
+                                 int B, int H, int N, int d, float sm_scale,
+                                 void *workspace, size_t workspace_bytes,
+                                 sage_stream_t stream,
+                                 sage_event_t attn_begin, sage_event_t attn_end);
 
 /*
  * sage_attn_dense_ref_gpu -- plain dense attention on the CUDA cores in fp32

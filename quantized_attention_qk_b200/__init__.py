@@ -23,6 +23,7 @@ __all__ = [
     "sage_quant_workspace_bytes", "sage_check", "sage_attn_fwd_host", "n_pad",
     "sage_block_select", "sage_attn_fwd_sparse", "sage_tau_schedule", "sage_block_mask_bytes",
     "sage_attn_sparse_workspace_bytes", "n_tiles", "mask_words", "mask_to_keep", "keep_to_mask",
+    "sage_attn_fwd_kres", "sage_quant_k_residual", "sage_attn_kres_workspace_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -68,6 +69,10 @@ _SIGS = {
     "sage_attn_fwd_sparse": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
                               ctypes.c_float, _P, _P, _P, _SZ, _P, _P, _P], _I32),
     "sage_tau_schedule": ([_I32, _I32, ctypes.c_float, ctypes.c_float], ctypes.c_float),
+    "sage_attn_kres_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_quant_k_residual": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
+    "sage_attn_fwd_kres": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                            _P, _SZ, _P, _P, _P], _I32),
 }
 
 
@@ -372,3 +377,43 @@ def sage_attn_fwd_sparse(q, k, v, tau=1.0, sm_scale=None, mask=None, return_mask
                                       ctypes.c_float(tau), _ptr(mask), _ptr(mask_out), _ptr(workspace), ws_bytes,
                                       _stream(stream, dev), e0, e1))
     return (out, mask_out) if return_mask else out
+
+
+# --------------------------------------------------------------------------
+# K-residual quantization (the sol-attn page's item 1; include/sage.h)
+# --------------------------------------------------------------------------
+
+def sage_attn_kres_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().sage_attn_kres_workspace_bytes(B, H, N, d))
+
+
+def sage_quant_k_residual(k, stream=None):
+    """Residual codes of K: dict k_i8 [B,H,N_pad,d] int8, k_scale [B,H,N_pad/64]
+    fp32, k_bmean [B,H,N_pad/64,d] bf16 bit patterns (int16 tensor)."""
+    _check_qkv(k)
+    B, H, N, d = k.shape
+    dev = k.device
+    npd = n_pad(N)
+    r = dict(k_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
+             k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
+             k_bmean=torch.empty(B, H, npd // K_BLOCK, d, dtype=torch.int16, device=dev))
+    _raise(lib().sage_quant_k_residual(_ptr(k), _strides(k), B, H, N, d, _ptr(r["k_i8"]), _ptr(r["k_scale"]),
+                                       _ptr(r["k_bmean"]), _stream(stream, dev)))
+    return r
+
+
+def sage_attn_fwd_kres(q, k, v, sm_scale=None, out=None, workspace=None, stream=None, attn_events=None):
+    """Quantized attention forward with K-residual quantization; returns bf16 [B,H,N,d]."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    dev = q.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
+    _raise(lib().sage_attn_fwd_kres(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                    _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                    _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
+    return out

@@ -401,6 +401,63 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], con
     return SAGE_OK;
 }
 
+static size_t kres_bmean_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.d * 2); }
+static size_t kres_ebias_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.n_pad() * 4); }
+
+size_t sage_attn_kres_workspace_bytes(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    const Shape s{B, H, N, d};
+    return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + kres_bmean_bytes(s) + kres_ebias_bytes(s);
+}
+
+sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4], int B, int H, int N, int d,
+                                    int8_t *k_i8, float *k_scale, uint16_t *k_bmean, sage_stream_t stream) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_view(k_bf16, k_stride, "k")) ||
+        (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(k_scale, "k_scale", 4)) ||
+        (r = check_dev(k_bmean, "k_bmean", 16)))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaError_t e = launch_kres(s, src(k_bf16, k_stride), k_i8, k_scale, k_bmean, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "K-residual quantization");
+    return SAGE_OK;
+}
+
+sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4], const void *k, const int64_t k_stride[4],
+                                 const void *v, const int64_t v_stride[4], void *out, const int64_t o_stride[4], int B,
+                                 int H, int N, int d, float sm_scale, void *workspace, size_t workspace_bytes,
+                                 sage_stream_t stream, sage_event_t attn_begin, sage_event_t attn_end) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
+        (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
+        (r = check_view(out, o_stride, "out")))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    const size_t cb = up(codes_bytes(s)), sb = up(stats_ws_bytes(s)), mb = kres_bmean_bytes(s);
+    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + sb + mb + kres_ebias_bytes(s), st))) return r;
+    char *base = static_cast<char *>(scr.ptr);
+    const Codes c = carve_codes(base, s);
+    const StatsWs ws = carve_stats_ws(base + cb, s);
+    uint16_t *bmean = reinterpret_cast<uint16_t *>(base + cb + sb);
+    float *ebias = reinterpret_cast<float *>(base + cb + sb + mb);
+    const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
+    cudaError_t e = launch_stats(s, nullptr, &vs, ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, &qs, nullptr, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if ((e = launch_kres(s, ks, c.k_i8, c.k_scale, bmean, st)) != cudaSuccess)
+        return cuda_fail(e, "K-residual quantization");
+    if ((e = launch_ebias(s, qs, bmean, sm_scale, ebias, st)) != cudaSuccess) return cuda_fail(e, "mean term");
+    if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_attention_kres(s, c, dst(out, o_stride), sm_scale, ebias, st)) != cudaSuccess)
+        return cuda_fail(e, "attention kernel");
+    if (attn_end && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_end), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    return SAGE_OK;
+}
+
 sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4], const void *k,
                                       const int64_t k_stride[4], const void *v, const int64_t v_stride[4], void *out,
                                       const int64_t o_stride[4], int B, int H, int N, int d, float sm_scale,

@@ -34,6 +34,11 @@
 // one shared load per role.  The producer streams the union through the ring;
 // each tile's QK and PV MMAs, barriers and P buffers advance with the tile's
 // own step count; a tile that keeps no key tile writes zeros.
+// K-residual instantiation (KRES): K holds the codes of its residual inside
+// each 64-token block, and every score gains that block's mean term e[row][b]
+// (precomputed in fp32, block-major so a warp's rows read it coalesced); each
+// 128-key step covers two blocks, so e folds into the two per-half offsets
+// the exponent already takes (no work per score).
 // Numerics (readings C4-C8): x = S*(sq*sm_scale*log2e*sk) with one sk per
 // 64-key block; running max m' = max(m, ceil(rowmax x)) so that the O / l
 // rescale 2^(m-m') is an exact power of two; P = e4m3(2^(x-m') * 448) computed as
@@ -117,6 +122,8 @@ struct AttnParams {
     // query tile i attends to key tile j
     const uint32_t *kv_mask;
     int mask_words;
+    // KRES instantiation: mean term of every (K block, query row), [BH][nkb][N_pad]
+    const float *ebias;
 };
 
 // Step lists of the SPARSE instantiation, built by one warp from mask rows r0
@@ -259,7 +266,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int D, bool EXPORT_S, bool SPARSE>
+template <int D, bool EXPORT_S, bool SPARSE, bool KRES>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
            const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
@@ -492,15 +499,25 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         float m = -INFINITY, l = 0.f;
         float ks_next0 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next);
         float ks_next1 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next + 1);
+        // KRES: this row's mean terms, [K block][row] with a row stride of N_pad
+        const int64_t npad = (int64_t)p.nqb * C::BM;
+        const float *eb = KRES ? p.ebias + (int64_t)bh * p.nkb * npad + grow : nullptr;
+        float e_next0 = KRES ? __ldg(eb + (2 * kt_next) * npad) : 0.f;
+        float e_next1 = KRES ? __ldg(eb + (2 * kt_next + 1) * npad) : 0.f;
         bool ok = true;
         for (int j = 0; ok && j < steps; ++j) {
             // this step's key tile and its two K-block scales were fetched one step ahead
             const int kt = kt_next;
             const float ks0 = ks_next0, ks1 = ks_next1;
+            const float e0 = e_next0, e1 = e_next1;
             if (!EXPORT_S && j + 1 < steps) {
                 kt_next = SPARSE ? mylist[j + 1] : j + 1;
                 ks_next0 = __ldg(ksc + 2 * kt_next);
                 ks_next1 = __ldg(ksc + 2 * kt_next + 1);
+                if (KRES) {
+                    e_next0 = __ldg(eb + (2 * kt_next) * npad);
+                    e_next1 = __ldg(eb + (2 * kt_next + 1) * npad);
+                }
             }
             if (!(ok = wait_warp(&ctl->s_full[t], j & 1, p.err, &ctl->abort, 10 + t))) break;
             tc_fence_after();
@@ -542,21 +559,23 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     x0 = mx0 == INT_MIN ? -INFINITY : static_cast<float>(mx0) * c0;
                     x1 = mx1 == INT_MIN ? -INFINITY : static_cast<float>(mx1) * c1;
                 }
+                if (KRES) x0 += e0, x1 += e1;
                 const float m_new = fmaxf(m, ceilf(fmaxf(x0, x1)));
                 const float alpha = (m == -INFINITY) ? 0.f : exp2_int(m - m_new);
                 const float nb = kLog2_448 - m_new;
+                const float nb0 = KRES ? nb + e0 : nb, nb1 = KRES ? nb + e1 : nb;
                 float acc[4] = {0.f, 0.f, 0.f, 0.f};
                 uint32_t w[32];
                 if (n_valid == C::BN) {
-                    p_pack32<false>(ra, c0, nb, 0, n_valid, acc, w + 0);
-                    p_pack32<false>(rb, c0, nb, 32, n_valid, acc, w + 8);
-                    p_pack32<false>(rc, c1, nb, 64, n_valid, acc, w + 16);
-                    p_pack32<false>(rd, c1, nb, 96, n_valid, acc, w + 24);
+                    p_pack32<false>(ra, c0, nb0, 0, n_valid, acc, w + 0);
+                    p_pack32<false>(rb, c0, nb0, 32, n_valid, acc, w + 8);
+                    p_pack32<false>(rc, c1, nb1, 64, n_valid, acc, w + 16);
+                    p_pack32<false>(rd, c1, nb1, 96, n_valid, acc, w + 24);
                 } else {
-                    p_pack32<true>(ra, c0, nb, 0, n_valid, acc, w + 0);
-                    p_pack32<true>(rb, c0, nb, 32, n_valid, acc, w + 8);
-                    p_pack32<true>(rc, c1, nb, 64, n_valid, acc, w + 16);
-                    p_pack32<true>(rd, c1, nb, 96, n_valid, acc, w + 24);
+                    p_pack32<true>(ra, c0, nb0, 0, n_valid, acc, w + 0);
+                    p_pack32<true>(rb, c0, nb0, 32, n_valid, acc, w + 8);
+                    p_pack32<true>(rc, c1, nb1, 64, n_valid, acc, w + 16);
+                    p_pack32<true>(rd, c1, nb1, 96, n_valid, acc, w + 24);
                 }
                 l = l * alpha + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
                 // P buffer j%2 was last read by PV(j-2), which finished before S(j)
@@ -690,7 +709,7 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
 }
 
 
-template <int D, bool EXPORT_S, bool SPARSE>
+template <int D, bool EXPORT_S, bool SPARSE, bool KRES = false>
 cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
                           const AttnParams &p0, dim3 grid, cudaStream_t st) {
     using C = Cfg<D>;
@@ -709,7 +728,7 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if (!p.err) return cudaErrorSymbolNotFound;
     const int smem = smem_bytes<D>(SPARSE ? 7 * p.nqb + 8 : 0);  // three uint16 lists and one uint8 list
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    auto kern = k_attn<D, EXPORT_S, SPARSE>;
+    auto kern = k_attn<D, EXPORT_S, SPARSE, KRES>;
     // The setmaxnreg split assumes the kernel is launched with LAUNCH_REGS per
     // thread; with fewer the increases could never be satisfied.
     cudaFuncAttributes fa;
@@ -781,6 +800,27 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
     return s.d == 128 ? launch_attn_d<128, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
                       : launch_attn_d<64, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
+}
+
+cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,
+                                  cudaStream_t st) {
+    AttnParams p{};
+    p.q_scale = c.q_scale;
+    p.k_scale = c.k_scale;
+    p.v_scale = c.v_scale;
+    p.out = out.p;
+    p.osb = out.sb;
+    p.osh = out.sh;
+    p.osn = out.sn;
+    p.H = s.H;
+    p.N = s.N;
+    p.nqb = s.n_qblocks();
+    p.nkb = s.n_kblocks();
+    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    p.ebias = ebias;
+    dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
+    return s.d == 128 ? launch_attn_d<128, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
+                      : launch_attn_d<64, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
 }
 
 cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,

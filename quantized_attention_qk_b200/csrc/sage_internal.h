@@ -87,6 +87,15 @@ unsigned *device_error_ptr();
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);
 cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,
                                     const uint32_t *kv_mask, cudaStream_t st);
+// K-residual mode: attention with the mean term ebias [BH][nkb][N_pad] added
+// to the scores (sage_attn.cu); the residual codes and the mean term
+// (sage_kres.cu).
+cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,
+                                  cudaStream_t st);
+cudaError_t launch_kres(const Shape &s, const Src &k, int8_t *k_i8, float *k_scale, uint16_t *k_bmean,
+                        cudaStream_t st);
+cudaError_t launch_ebias(const Shape &s, const Src &q, const uint16_t *k_bmean, float sm_scale, float *ebias,
+                         cudaStream_t st);
 cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,
                                  int kv_tile, int32_t *s_out, cudaStream_t st);
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st);

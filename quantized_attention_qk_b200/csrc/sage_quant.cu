@@ -510,6 +510,7 @@ cudaError_t launch_quant_d(const Shape &s, const Src *q, const Src *k, const Src
     if (q && k && !v) return launch_quant_k<D, true, true, false>(s, tq, tk, tv, a, st);
     if (!q && k && v) return launch_quant_k<D, false, true, true>(s, tq, tk, tv, a, st);
     if (!q && !k && v) return launch_quant_k<D, false, false, true>(s, tq, tk, tv, a, st);
+    if (q && !k && v) return launch_quant_k<D, true, false, true>(s, tq, tk, tv, a, st);
     return cudaErrorInvalidValue;
 }
 
