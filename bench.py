@@ -208,6 +208,9 @@ def run_gpu(args):
             if args.kres:
                 return sage.sage_attn_fwd_kres(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws,
                                                attn_events=events)
+            if args.fused_q:
+                return sage.sage_attn_fwd_fused_q(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws,
+                                                  attn_events=events)
             return sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale, out=out, workspace=ws, attn_events=events)
 
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
@@ -282,7 +285,7 @@ def run_gpu(args):
                    "l2": "flushed before every timed step (256 MB write, outside the events)"},
         "roofline": {"bound": "tensor", "kernel": "k_attn (fused attention)", "achieved": round(attn_tops, 2),
                      "peak": round(peak_8bit, 1), "unit": "TFLOP/s", "frac": round(attn_tops / peak_8bit, 4),
-                     "traffic": None if (args.tau is not None or args.kres) else _attn_traffic(wp.name),
+                     "traffic": None if (args.tau is not None or args.kres or args.fused_q) else _attn_traffic(wp.name),
                      "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
@@ -298,10 +301,12 @@ def run_gpu(args):
         line["config"]["kept_fraction"] = round(r["kept"], 4)
         line["config"]["ops"] = ("value counts the dense 4*B*H*N^2*d; roofline.achieved counts the kept tile "
                                  "pairs only (block-sparse forward, sage_attn_fwd_sparse)")
+    if args.fused_q:
+        line["config"]["q_quantization"] = "in the attention kernel's prologue (sage_attn_fwd_fused_q)"
     if args.kres:
         line["config"]["k_residual"] = ("K-residual quantization (sage_attn_fwd_kres): residual codes per 64-token "
                                         "block, bf16 block means, mean term on the tensor cores")
-    if args.secondary and args.workload != SECONDARY and args.tau is None and not args.kres:
+    if args.secondary and args.workload != SECONDARY and args.tau is None and not args.kres and not args.fused_q:
         ws_ = WORKLOADS[SECONDARY]
         r2 = measure(ws_, max(3, args.steps // 2), args.warmup)
         k2 = max(3, args.steps // 2)
@@ -364,6 +369,8 @@ def main():
                     help="time the block-sparse forward with this tau instead of the dense one")
     ap.add_argument("--kres", action="store_true",
                     help="time the K-residual forward instead of the smoothing one")
+    ap.add_argument("--fused-q", dest="fused_q", action="store_true",
+                    help="time the forward that quantizes Q in the attention kernel's prologue")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -306,6 +306,23 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4],
  */
 float sage_tau_schedule(int step, int n_steps, float tau_start, float tau_end);
 
+/*
+ * sage_attn_fwd_fused_q -- sage_attn_fwd with Q quantized inside the fused
+ * attention kernel: the quantize pass codes K and V only; each attention CTA
+ * loads its two tiles' bf16 Q rows, takes each tile's |max| and writes the
+ * INT8 codes into shared memory with the same arithmetic, so the result equals
+ * sage_attn_fwd's bit for bit.  Same arguments, scratch size
+ * (sage_attn_workspace_bytes), events and errors as sage_attn_fwd_ev.
+ */
+sage_status_t sage_attn_fwd_fused_q(const void *q, const int64_t q_stride[4],
+                                    const void *k, const int64_t k_stride[4],
+                                    const void *v, const int64_t v_stride[4],
+                                    void *out, const int64_t o_stride[4],
+                                    int B, int H, int N, int d, float sm_scale,
+                                    void *workspace, size_t workspace_bytes,
+                                    sage_stream_t stream,
+                                    sage_event_t attn_begin, sage_event_t attn_end);
+
 /* ------------------------------------------------------------------------ */
 /* K-residual quantization ([SOL] item 1: quantize only the residual of K     */
 /* inside each block; keep the block-mean term at bf16 precision).  Readings  */

@@ -23,7 +23,7 @@ __all__ = [
     "sage_quant_workspace_bytes", "sage_check", "sage_attn_fwd_host", "n_pad",
     "sage_block_select", "sage_attn_fwd_sparse", "sage_tau_schedule", "sage_block_mask_bytes",
     "sage_attn_sparse_workspace_bytes", "n_tiles", "mask_words", "mask_to_keep", "keep_to_mask",
-    "sage_attn_fwd_kres", "sage_quant_k_residual", "sage_attn_kres_workspace_bytes",
+    "sage_attn_fwd_kres", "sage_quant_k_residual", "sage_attn_kres_workspace_bytes", "sage_attn_fwd_fused_q",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +70,8 @@ _SIGS = {
                               ctypes.c_float, _P, _P, _P, _SZ, _P, _P, _P], _I32),
     "sage_tau_schedule": ([_I32, _I32, ctypes.c_float, ctypes.c_float], ctypes.c_float),
     "sage_attn_kres_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_attn_fwd_fused_q": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
+                               _P, _SZ, _P, _P, _P], _I32),
     "sage_quant_k_residual": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
     "sage_attn_fwd_kres": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
                             _P, _SZ, _P, _P, _P], _I32),
@@ -416,4 +418,22 @@ def sage_attn_fwd_kres(q, k, v, sm_scale=None, out=None, workspace=None, stream=
     _raise(lib().sage_attn_fwd_kres(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                     _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
                                     _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
+    return out
+
+
+def sage_attn_fwd_fused_q(q, k, v, sm_scale=None, out=None, workspace=None, stream=None, attn_events=None):
+    """sage_attn_fwd with Q quantized in the attention kernel's prologue (the
+    same result bit for bit); returns bf16 [B,H,N,d]."""
+    _check_qkv(q, k, v)
+    B, H, N, d = q.shape
+    dev = q.device
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
+    _raise(lib().sage_attn_fwd_fused_q(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+                                       _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
+                                       _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
     return out

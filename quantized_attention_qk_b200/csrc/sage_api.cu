@@ -401,6 +401,36 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], con
     return SAGE_OK;
 }
 
+sage_status_t sage_attn_fwd_fused_q(const void *q, const int64_t q_stride[4], const void *k,
+                                   const int64_t k_stride[4], const void *v, const int64_t v_stride[4], void *out,
+                                   const int64_t o_stride[4], int B, int H, int N, int d, float sm_scale,
+                                   void *workspace, size_t workspace_bytes, sage_stream_t stream,
+                                   sage_event_t attn_begin, sage_event_t attn_end) {
+    sage_status_t r;
+    if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
+        (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
+        (r = check_view(out, o_stride, "out")))
+        return r;
+    const Shape s{B, H, N, d};
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    Scratch scr;
+    const size_t cb = up(codes_bytes(s));
+    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + stats_ws_bytes(s), st))) return r;
+    const Codes c = carve_codes(scr.ptr, s);
+    const StatsWs ws = carve_stats_ws(static_cast<char *>(scr.ptr) + cb, s);
+    const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
+    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
+    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
+    if ((e = launch_quant(s, nullptr, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    if ((e = launch_attention_fused_q(s, c, qs, dst(out, o_stride), sm_scale, st)) != cudaSuccess)
+        return cuda_fail(e, "attention kernel");
+    if (attn_end && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_end), st)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    return SAGE_OK;
+}
+
 static size_t kres_bmean_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.d * 2); }
 static size_t kres_ebias_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.n_pad() * 4); }
 

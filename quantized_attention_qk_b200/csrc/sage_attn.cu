@@ -34,6 +34,13 @@
 // one shared load per role.  The producer streams the union through the ring;
 // each tile's QK and PV MMAs, barriers and P buffers advance with the tile's
 // own step count; a tile that keeps no key tile writes zeros.
+// Prologue-quantized Q (FUSED_Q): the producer loads the bf16 rows of both
+// tiles into the P buffers (idle until the first P is stored); each softmax
+// warpgroup takes its tile's |max| (each thread its row, the four warps
+// combined through shared memory) and codes the rows into the swizzled INT8
+// Q tile with the quantize pass's arithmetic, so the codes are the same and
+// the quantize pass codes K and V only.  No P is stored before S(0), which
+// waits for all eight warps' codes.
 // K-residual instantiation (KRES): K holds the codes of its residual inside
 // each 64-token block, and every score gains that block's mean term e[row][b]
 // (precomputed in fp32, block-major so a warp's rows read it coalesced); each
@@ -92,6 +99,9 @@ struct Ctl {
     uint64_t o_done[2];     // per tile: PV of a step completed
     uint64_t o_final[2];    // per tile: every PV of the tile completed (committed once)
     uint64_t drain;
+    uint64_t qb_full;       // FUSED_Q: the bf16 Q rows landed
+    uint64_t q_amax_bar[2]; // FUSED_Q, per tile: the four warps posted their |max|
+    float q_amax[2][4];
     int steps[3];           // SPARSE: own steps of tile 0, of tile 1, union steps
     uint32_t tmem_base;
     AbortState abort;
@@ -124,6 +134,7 @@ struct AttnParams {
     int mask_words;
     // KRES instantiation: mean term of every (K block, query row), [BH][nkb][N_pad]
     const float *ebias;
+    int q_swap;            // FUSED_Q: the bf16 Q map takes H before N
 };
 
 // Step lists of the SPARSE instantiation, built by one warp from mask rows r0
@@ -266,10 +277,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
-template <int D, bool EXPORT_S, bool SPARSE, bool KRES>
+template <int D, bool EXPORT_S, bool SPARSE, bool KRES, bool FUSED_Q>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-           const __grid_constant__ CUtensorMap tm_v, const AttnParams p) {
+           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qb, const AttnParams p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -290,7 +301,10 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     const int nkv = EXPORT_S ? 1 : (p.N + C::BN - 1) / C::BN;
 
     if (threadIdx.x == 0) {
-        mbar_init(&ctl->q_full, 1);
+        mbar_init(&ctl->q_full, FUSED_Q ? 8 : 1);  // the softmax warps' codes, or the TMA
+        mbar_init(&ctl->qb_full, 1);
+        mbar_init(&ctl->q_amax_bar[0], 4);
+        mbar_init(&ctl->q_amax_bar[1], 4);
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(&ctl->kv_full[s], 1);
             mbar_init(&ctl->kv_empty[s], 1);
@@ -308,7 +322,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         fence_barrier_init();
     }
     if (warp == 8 && lane == 0) {
-        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(FUSED_Q ? &tm_qb : &tm_q);
         tma_prefetch_desc(&tm_k);
         if (!EXPORT_S) tma_prefetch_desc(&tm_v);
     }
@@ -337,9 +351,25 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     if (warp == 8) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            mbar_arrive_expect_tx(&ctl->q_full, 2 * C::Q_BYTES);
-            tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, qt0 * C::BM, bh);
-            tma_load_3d(sQ + C::Q_BYTES, &tm_q, &ctl->q_full, 0, (qt0 + 1) * C::BM, bh);
+            if (FUSED_Q) {
+                // bf16 rows of both tiles into the P buffers: [tile][d/64][128 rows][64]
+                const int b = bh / p.H, h = bh % p.H;
+                mbar_arrive_expect_tx(&ctl->qb_full, 2 * C::BM * D * 2);
+                for (int t = 0; t < 2; ++t)
+                    for (int half = 0; half < D / 64; ++half)
+                        for (int r = 0; r < C::BM; r += 64) {
+                            uint16_t *dst = reinterpret_cast<uint16_t *>(sP) + ((t * (D / 64) + half) * C::BM + r) * 64;
+                            const int n = (qt0 + t) * C::BM + r;
+                            if (p.q_swap)
+                                tma_load_4d(dst, &tm_qb, &ctl->qb_full, half * 64, h, n, b);
+                            else
+                                tma_load_4d(dst, &tm_qb, &ctl->qb_full, half * 64, n, h, b);
+                        }
+            } else {
+                mbar_arrive_expect_tx(&ctl->q_full, 2 * C::Q_BYTES);
+                tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, qt0 * C::BM, bh);
+                tma_load_3d(sQ + C::Q_BYTES, &tm_q, &ctl->q_full, 0, (qt0 + 1) * C::BM, bh);
+            }
             int issued = 0;
             const int nsteps = SPARSE ? ctl->steps[2] : nkv;
             for (int j = 0; j < nsteps; ++j) {
@@ -355,7 +385,7 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 issued = j + 1;
             }
             // every copy started here lands before the CTA may exit
-            wait_one(&ctl->q_full, 0, p.err, &ctl->abort, true, 2);
+            wait_one(FUSED_Q ? &ctl->qb_full : &ctl->q_full, 0, p.err, &ctl->abort, true, 2);
             for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
                 wait_one(&ctl->kv_full[j % C::STAGES], (j / C::STAGES) & 1, p.err, &ctl->abort, true, 3);
         }
@@ -489,7 +519,61 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         const uint32_t tS = tmem + lane_off + t * 128;
         const uint32_t tO = tmem + lane_off + C::T_O + t * D;
         const uint32_t pbase = smem_u32(sP) + 2 * t * C::P_BYTES;
-        const float sq = qt < p.nqb ? p.q_scale[(int64_t)bh * p.nqb + qt] : 0.f;
+        bool ok = true;
+        float sq;
+        if constexpr (FUSED_Q) {
+            // This tile's bf16 rows are in the P buffers; the tile's block scale is
+            // its |max| / 127 and the codes rne(x * fp32(127 / |max|)).  Each warp
+            // takes its own 32 rows four at a time: lane l holds the 8 channels
+            // 8 (l mod 8).. of row 4i + l/8 in each 64-channel half, so a warp's
+            // 16-byte loads cover four whole 128-byte rows (no bank conflicts).
+            const uint16_t *qtile = reinterpret_cast<const uint16_t *>(sP) + t * (D / 64) * C::BM * 64;
+            float amax = 0.f;
+            if ((ok = wait_warp(&ctl->qb_full, 0, p.err, &ctl->abort, 14))) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int half = 0; half < D / 64; ++half) {
+                        const int r = wq * 32 + i * 4 + (lane >> 3);
+                        float f[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(qtile + (half * C::BM + r) * 64 + (lane & 7) * 8), f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+                    }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                if (lane == 0) ctl->q_amax[t][wq] = amax;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->q_amax_bar[t]);
+                ok = wait_warp(&ctl->q_amax_bar[t], 0, p.err, &ctl->abort, 14);
+            }
+            if (ok) {
+                amax = fmaxf(fmaxf(ctl->q_amax[t][0], ctl->q_amax[t][1]), fmaxf(ctl->q_amax[t][2], ctl->q_amax[t][3]));
+                const float inv = amax > 0.f ? __fdiv_rn(127.f, amax) : 0.f;
+                // codes at their swizzled places in the K-major tile (128-byte
+                // swizzle for d = 128, 64-byte for d = 64, as the TMA writes them):
+                // 16-byte chunk c of row r sits at r*d + ((c ^ swz(r)) * 16)
+                const uint32_t qdst = smem_u32(sQ + t * C::Q_BYTES);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+#pragma unroll
+                    for (int half = 0; half < D / 64; ++half) {
+                        const int r = wq * 32 + i * 4 + (lane >> 3);
+                        const int ch = half * 64 + (lane & 7) * 8;  // first of this lane's 8 channels
+                        float f[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(qtile + (half * C::BM + r) * 64 + (lane & 7) * 8), f);
+                        const uint2 w = i8x8(f, inv);
+                        const int swz = D == 128 ? (r & 7) : ((r >> 1) & 3);
+                        st_shared_v2(qdst + r * D + (((ch >> 4) ^ swz) << 4) + ((ch >> 3) & 1) * 8, w.x, w.y);
+                    }
+                fence_proxy_async_smem();  // make the codes visible to the tensor core
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->q_full);
+            }
+            sq = amax > 0.f ? __fdiv_rn(amax, 127.f) : 0.f;
+        } else {
+            sq = qt < p.nqb ? p.q_scale[(int64_t)bh * p.nqb + qt] : 0.f;
+        }
         const float cq = sq * p.s_l2;
         const float kLog2_448 = 8.807354922057604f;
         const float *ksc = p.k_scale + (int64_t)bh * p.nkb + 2 * kv0;
@@ -504,7 +588,6 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         const float *eb = KRES ? p.ebias + (int64_t)bh * p.nkb * npad + grow : nullptr;
         float e_next0 = KRES ? __ldg(eb + (2 * kt_next) * npad) : 0.f;
         float e_next1 = KRES ? __ldg(eb + (2 * kt_next + 1) * npad) : 0.f;
-        bool ok = true;
         for (int j = 0; ok && j < steps; ++j) {
             // this step's key tile and its two K-block scales were fetched one step ahead
             const int kt = kt_next;
@@ -709,13 +792,19 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
 }
 
 
-template <int D, bool EXPORT_S, bool SPARSE, bool KRES = false>
+template <int D, bool EXPORT_S, bool SPARSE, bool KRES = false, bool FUSED_Q = false>
 cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
-                          const AttnParams &p0, dim3 grid, cudaStream_t st) {
+                          const AttnParams &p0, dim3 grid, cudaStream_t st, const Src *q_bf16 = nullptr) {
     using C = Cfg<D>;
     const int n_pad = s.n_pad();
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, tqb;
+    AttnParams p = p0;
     cudaError_t e;
+    if (FUSED_Q) {
+        if (!q_bf16) return cudaErrorInvalidValue;
+        if ((e = make_bf16_token_map(&tqb, *q_bf16, s, 64, &p.q_swap)) != cudaSuccess) return e;
+        q_i8 = k_i8;  // the INT8 Q map is not read; any valid map will do
+    }
     if ((e = make_map(&tq, q_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BM)) != cudaSuccess) return e;
     if ((e = make_map(&tk, k_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) return e;
     if (EXPORT_S) {
@@ -723,19 +812,19 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     } else if ((e = make_map(&tv, v_e4m3, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) {
         return e;
     }
-    AttnParams p = p0;
+    if (!FUSED_Q) tqb = tq;  // not read
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorSymbolNotFound;
     const int smem = smem_bytes<D>(SPARSE ? 7 * p.nqb + 8 : 0);  // three uint16 lists and one uint8 list
     if (smem > 227 * 1024) return cudaErrorInvalidValue;
-    auto kern = k_attn<D, EXPORT_S, SPARSE, KRES>;
+    auto kern = k_attn<D, EXPORT_S, SPARSE, KRES, FUSED_Q>;
     // The setmaxnreg split assumes the kernel is launched with LAUNCH_REGS per
     // thread; with fewer the increases could never be satisfied.
     cudaFuncAttributes fa;
     if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
     if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, smem, st>>>(tq, tk, tv, p);
+    kern<<<grid, C::THREADS, smem, st>>>(tq, tk, tv, tqb, p);
     return cudaGetLastError();
 }
 
@@ -800,6 +889,26 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
     return s.d == 128 ? launch_attn_d<128, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
                       : launch_attn_d<64, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
+}
+
+cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &q_bf16, const Dst &out,
+                                     float sm_scale, cudaStream_t st) {
+    AttnParams p{};
+    p.k_scale = c.k_scale;
+    p.v_scale = c.v_scale;
+    p.out = out.p;
+    p.osb = out.sb;
+    p.osh = out.sh;
+    p.osn = out.sn;
+    p.H = s.H;
+    p.N = s.N;
+    p.nqb = s.n_qblocks();
+    p.nkb = s.n_kblocks();
+    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
+    return s.d == 128
+               ? launch_attn_d<128, false, false, false, true>(s, nullptr, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16)
+               : launch_attn_d<64, false, false, false, true>(s, nullptr, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16);
 }
 
 cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,

@@ -87,6 +87,10 @@ unsigned *device_error_ptr();
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);
 cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,
                                     const uint32_t *kv_mask, cudaStream_t st);
+// Q quantized in the attention kernel's prologue from the bf16 view q_bf16
+// (c.q_i8 / c.q_scale are not used).
+cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &q_bf16, const Dst &out,
+                                     float sm_scale, cudaStream_t st);
 // K-residual mode: attention with the mean term ebias [BH][nkb][N_pad] added
 // to the scores (sage_attn.cu); the residual codes and the mean term
 // (sage_kres.cu).

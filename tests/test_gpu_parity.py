@@ -206,9 +206,9 @@ def test_fused_and_contiguous_layouts_give_identical_bits():
 
 @pytest.mark.parametrize("N,d,layout", [(4608, 128, "fused"), (1000, 128, "contiguous"), (200, 64, "contiguous"),
                                          (777, 64, "fused"), (129, 128, "fused"), (1, 64, "contiguous")])
-def test_prologue_q_quantization_matches_the_quantize_pass(N, d, layout):
-    """The forward quantizes Q inside the attention kernel; its output must be
-    bit-identical to the explicit path (quantize pass codes -> attention)."""
+def test_forward_matches_the_explicit_quantize_then_attention_path(N, d, layout):
+    """sage_attn_fwd against its own steps called one by one through the C ABI
+    (sage_quant_qk, sage_quant_v, sage_attn_quantized): the same bits."""
     w = tiny_custom(1, 3, N, d, seed=40 + N, layout=layout, bias_sigma=4.0, outlier_frac=0.01)
     _, (qd, kd, vd), _ = _inputs(w)
     fused = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
@@ -224,7 +224,7 @@ def test_prologue_q_quantization_matches_the_quantize_pass(N, d, layout):
 @pytest.mark.parametrize("B,H,N,d,layout,pinned", [(1, 24, 1000, 128, "fused", True), (2, 5, 777, 64, "contiguous", True),
                                                    (2, 3, 300, 128, "fused", False), (1, 1, 129, 64, "fused", True)])
 def test_host_memory_forward_matches_the_device_forward(B, H, N, d, layout, pinned):
-    """sage_attn_fwd_host (head chunks on two streams, host<->device copies
+    """sage_attn_fwd_host (head chunks on three streams, host<->device copies
     inside) gives the device forward's bits."""
     w = tiny_custom(B, H, N, d, seed=70 + N, layout=layout, bias_sigma=4.0, outlier_frac=0.01)
     _, (qd, kd, vd), bufs = _inputs(w)
@@ -318,3 +318,21 @@ def test_quantized_against_exact_is_the_schemes_own_error():
 
 def test_device_error_word_is_clear():
     sage.sage_check()
+
+
+@pytest.mark.parametrize("w", [
+    WORKLOADS["tiny"],
+    tiny_custom(1, 2, 300, 64, 701, layout="fused", bias_sigma=2.0),
+    tiny_custom(2, 3, 777, 128, 702, bias_sigma=4.0, outlier_frac=0.01),
+    tiny_custom(1, 1, 50, 128, 703, layout="fused"),
+    WORKLOADS["flux"],
+], ids=lambda w: w.name)
+def test_prologue_q_quantization_forward_is_bit_identical(w):
+    """sage_attn_fwd_fused_q (Q coded inside the attention kernel) against the
+    forward with the quantize pass coding Q: the same codes, so the same bits."""
+    _, (qd, kd, vd), _ = _inputs(w)
+    ref = sage.sage_attn_fwd(qd, kd, vd, sm_scale=w.sm_scale)
+    got = sage.sage_attn_fwd_fused_q(qd, kd, vd, sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    assert torch.equal(got, ref)
