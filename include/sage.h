@@ -390,6 +390,16 @@ sage_status_t sage_debug_qk_tile(const int8_t *q_i8, const int8_t *k_i8,
                                  int b, int h, int q_tile, int kv_tile,
                                  int32_t *s_out, sage_stream_t stream);
 
+/*
+ * sage_debug_wait_timeout -- a probe of the failure path every kernel uses:
+ * one warp waits, bounded to `microseconds` (1..1000000) of SM clocks, on a
+ * barrier that nothing arrives on, gives up, records the timeout in the
+ * device error word (bit 0 and bit 8 + site 0) and returns normally.  The
+ * next sage_check on the stream reports SAGE_ERR_TIMEOUT and clears the word;
+ * the context stays usable.  Nothing faults, traps or hangs.
+ */
+sage_status_t sage_debug_wait_timeout(int microseconds, sage_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -70,6 +70,7 @@ _SIGS = {
                               ctypes.c_float, _P, _P, _P, _SZ, _P, _P, _P], _I32),
     "sage_tau_schedule": ([_I32, _I32, ctypes.c_float, ctypes.c_float], ctypes.c_float),
     "sage_attn_kres_workspace_bytes": ([_I32] * 4, _SZ),
+    "sage_debug_wait_timeout": ([_I32, _P], _I32),
     "sage_attn_fwd_fused_q": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
                                _P, _SZ, _P, _P, _P], _I32),
     "sage_quant_k_residual": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
@@ -437,3 +438,10 @@ def sage_attn_fwd_fused_q(q, k, v, sm_scale=None, out=None, workspace=None, stre
                                        _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
                                        _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
     return out
+
+
+def sage_debug_wait_timeout(microseconds: int = 10000, stream=None, device=None):
+    """Launch the bounded-wait probe (include/sage.h): the next sage_check on
+    the stream reports SAGE_ERR_TIMEOUT."""
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _raise(lib().sage_debug_wait_timeout(int(microseconds), _stream(stream, dev)))

@@ -79,13 +79,12 @@ __device__ __forceinline__ bool wait_one(uint64_t *bar, uint32_t parity, unsigne
 // Warp-uniform bounded wait: every lane of the warp returns the same value,
 // so .sync.aligned instructions that follow stay convergent.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, unsigned *err_word,
-                                          AbortState *st, int site = 0) {
+                                          AbortState *st, int site = 0, long long limit = kWaitLimitClocks) {
     long long t0 = clock64();
     while (true) {
         bool ok = mbar_try_wait(bar, parity);
         if (__all_sync(0xffffffffu, ok)) return true;
-        bool give_up = *reinterpret_cast<volatile int *>(&st->flag) != 0 ||
-                       (clock64() - t0 > kWaitLimitClocks);
+        bool give_up = *reinterpret_cast<volatile int *>(&st->flag) != 0 || (clock64() - t0 > limit);
         if (__any_sync(0xffffffffu, give_up)) {
             if ((threadIdx.x & 31) == 0 && !*reinterpret_cast<volatile int *>(&st->flag))
                 record_timeout(err_word, st, site);

@@ -157,3 +157,9 @@ def test_mask_packing_round_trips():
         # bit j of word j // 32
         j = T - 1
         assert bool(((m[0, 0, 0, j // 32].item() & 0xFFFFFFFF) >> (j % 32)) & 1) == bool(keep[0, 0, 0, j])
+
+
+def test_wait_probe_rejects_out_of_range_limits_before_any_launch(L):
+    for us in (0, -5, 1000001):
+        assert L.sage_debug_wait_timeout(us, None) == 1
+        assert "microseconds" in L.sage_last_error_message().decode()
