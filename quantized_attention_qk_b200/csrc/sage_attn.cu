@@ -872,7 +872,9 @@ cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, 
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st) {
+// Parameters every attention launch shares: codes' scales, output view, shape
+// and fp32(sm_scale * fp32(log2 e)).
+AttnParams attn_params(const Shape &s, const Codes &c, const Dst &out, float sm_scale) {
     AttnParams p{};
     p.q_scale = c.q_scale;
     p.k_scale = c.k_scale;
@@ -886,6 +888,11 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
     p.nqb = s.n_qblocks();
     p.nkb = s.n_kblocks();
     p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    return p;
+}
+
+cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st) {
+    AttnParams p = attn_params(s, c, out, sm_scale);
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
     return s.d == 128 ? launch_attn_d<128, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
                       : launch_attn_d<64, false, false>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
@@ -893,18 +900,8 @@ cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, flo
 
 cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &q_bf16, const Dst &out,
                                      float sm_scale, cudaStream_t st) {
-    AttnParams p{};
-    p.k_scale = c.k_scale;
-    p.v_scale = c.v_scale;
-    p.out = out.p;
-    p.osb = out.sb;
-    p.osh = out.sh;
-    p.osn = out.sn;
-    p.H = s.H;
-    p.N = s.N;
-    p.nqb = s.n_qblocks();
-    p.nkb = s.n_kblocks();
-    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    AttnParams p = attn_params(s, c, out, sm_scale);
+    p.q_scale = nullptr;  // the kernel computes each tile's Q scale
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
     return s.d == 128
                ? launch_attn_d<128, false, false, false, true>(s, nullptr, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16)
@@ -913,19 +910,7 @@ cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &
 
 cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,
                                   cudaStream_t st) {
-    AttnParams p{};
-    p.q_scale = c.q_scale;
-    p.k_scale = c.k_scale;
-    p.v_scale = c.v_scale;
-    p.out = out.p;
-    p.osb = out.sb;
-    p.osh = out.sh;
-    p.osn = out.sn;
-    p.H = s.H;
-    p.N = s.N;
-    p.nqb = s.n_qblocks();
-    p.nkb = s.n_kblocks();
-    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    AttnParams p = attn_params(s, c, out, sm_scale);
     p.ebias = ebias;
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
     return s.d == 128 ? launch_attn_d<128, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
@@ -934,19 +919,7 @@ cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out
 
 cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,
                                     const uint32_t *kv_mask, cudaStream_t st) {
-    AttnParams p{};
-    p.q_scale = c.q_scale;
-    p.k_scale = c.k_scale;
-    p.v_scale = c.v_scale;
-    p.out = out.p;
-    p.osb = out.sb;
-    p.osh = out.sh;
-    p.osn = out.sn;
-    p.H = s.H;
-    p.N = s.N;
-    p.nqb = s.n_qblocks();
-    p.nkb = s.n_kblocks();
-    p.s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
+    AttnParams p = attn_params(s, c, out, sm_scale);
     p.kv_mask = kv_mask;
     p.mask_words = s.mask_words();
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
