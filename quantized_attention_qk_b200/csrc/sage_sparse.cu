@@ -24,8 +24,8 @@ namespace sage {
 namespace {
 
 constexpr int kPoolThreads = 256;  // 8 warps, each over every 8th row of a tile
-constexpr int kScoreTile = 32;     // k_score: 32 query tiles x 32 key tiles per CTA
-constexpr int kScoreThreads = 256; // each thread: one query tile x 4 key tiles
+constexpr int kScoreTile = 16;     // k_score: 16 query tiles x 16 key tiles per CTA
+constexpr int kScoreThreads = 256; // one (query tile, key tile) pair per thread
 constexpr int kSelThreads = 256;
 
 // Per (b,h, tile i): qv[i][c] = q_scale[i] * float(sum of the tile's Q codes
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(kPoolThreads)
     }
 }
 
-// Tile-pair scores (reading S2) for a 32 x 32 block of (query tile, key tile)
+// Tile-pair scores (reading S2) for a 16 x 16 block of (query tile, key tile)
 // pairs of one (b,h): both pooled operands staged in shared memory, each dot
 // product accumulated over the channels in ascending order, one fp32 rounding
 // per multiply and per add (no contraction), then * s_l2 / (n_i n_j).
@@ -100,31 +100,23 @@ __global__ void __launch_bounds__(kScoreThreads)
     __shared__ float sq[kScoreTile][D + 1];   // [query tile][channel]
     __shared__ float sk[D][kScoreTile];       // [channel][key tile]
     const int i0 = blockIdx.x * kScoreTile, j0 = blockIdx.y * kScoreTile, bh = blockIdx.z;
-    for (int x = threadIdx.x; x < kScoreTile * D; x += kScoreThreads) {
+    static_assert(kScoreTile * D % kScoreThreads == 0, "staging loop has a fixed trip count");
+#pragma unroll
+    for (int x = threadIdx.x; x < kScoreTile * D; x += kScoreThreads) {  // all loads in flight at once
         const int r = x / D, c = x - r * D;
         sq[r][c] = i0 + r < nt ? qv[((size_t)bh * nt + i0 + r) * D + c] : 0.f;
         const int cc = x / kScoreTile, jj = x - cc * kScoreTile;
         sk[cc][jj] = j0 + jj < nt ? kvT[((size_t)bh * D + cc) * nt + j0 + jj] : 0.f;
     }
     __syncthreads();
-    const int il = threadIdx.x >> 3, jl = (threadIdx.x & 7) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-        const float a = sq[il][c];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[e] = __fadd_rn(acc[e], __fmul_rn(a, sk[c][jl + e]));
-    }
-    const int i = i0 + il;
-    if (i >= nt) return;
-    const int ni = min(kKvTile, N - i * kKvTile);
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-        const int j = j0 + jl + e;
-        if (j >= nt) continue;
-        const int nj = min(kKvTile, N - j * kKvTile);
-        sbar[((size_t)bh * nt + i) * nt + j] = __fdiv_rn(__fmul_rn(acc[e], s_l2), static_cast<float>(ni * nj));
-    }
+    const int il = threadIdx.x / kScoreTile, jl = threadIdx.x % kScoreTile;
+    float acc = 0.f;
+#pragma unroll 16
+    for (int c = 0; c < D; ++c) acc = __fadd_rn(acc, __fmul_rn(sq[il][c], sk[c][jl]));
+    const int i = i0 + il, j = j0 + jl;
+    if (i >= nt || j >= nt) return;
+    const int ni = min(kKvTile, N - i * kKvTile), nj = min(kKvTile, N - j * kKvTile);
+    sbar[((size_t)bh * nt + i) * nt + j] = __fdiv_rn(__fmul_rn(acc, s_l2), static_cast<float>(ni * nj));
 }
 
 // One CTA per (b,h, query tile i): ranks the row's key tiles (bitonic sort of
@@ -139,7 +131,6 @@ __global__ void __launch_bounds__(kSelThreads)
     float *key = sm;                                       // [P] score, then mass
     int *idx = reinterpret_cast<int *>(key + P);           // [P] key tile
     uint32_t *mw = reinterpret_cast<uint32_t *>(idx + P);  // [words]
-    __shared__ float part[kSelThreads];
     const int i = blockIdx.x, bh = blockIdx.y;
     const float *row = sbar + ((size_t)bh * nt + i) * nt;
     for (int w = threadIdx.x; w < words; w += kSelThreads) mw[w] = 0u;
@@ -180,14 +171,24 @@ __global__ void __launch_bounds__(kSelThreads)
             key[r] = w;
             own += w;
         }
-        part[threadIdx.x] = own;
-        __syncthreads();
+        // exclusive scan of the thread sums in thread order: within each warp by
+        // shuffles, then over the warp totals
+        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+        float incl = own;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d) incl += o;
+        }
+        __shared__ float wsum[kSelThreads / 32];
         __shared__ float s_total;
-        if (threadIdx.x == 0) {  // exclusive scan of the thread sums, in thread order
+        if (lane == 31) wsum[wid] = incl;
+        __syncthreads();
+        if (threadIdx.x == 0) {
             float run = 0.f;
-            for (int t = 0; t < kSelThreads; ++t) {
-                const float v = part[t];
-                part[t] = run;
+            for (int w = 0; w < kSelThreads / 32; ++w) {
+                const float v = wsum[w];
+                wsum[w] = run;
                 run += v;
             }
             s_total = run;
@@ -195,7 +196,7 @@ __global__ void __launch_bounds__(kSelThreads)
         __syncthreads();
         // rank r is kept iff the mass ranked before it is below tau of the total
         const float lim = tau * s_total;
-        float before = part[threadIdx.x];
+        float before = wsum[wid] + (incl - own);
         for (int r = r0; r < r1 && before < lim; ++r) {
             const int j = idx[r];
             atomicOr(&mw[j >> 5], 1u << (j & 31));
