@@ -163,3 +163,14 @@ def test_wait_probe_rejects_out_of_range_limits_before_any_launch(L):
     for us in (0, -5, 1000001):
         assert L.sage_debug_wait_timeout(us, None) == 1
         assert "microseconds" in L.sage_last_error_message().decode()
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No library, no result: the binding raises instead of computing anything
+    another way."""
+    monkeypatch.setattr(sage, "LIB_PATH", str(tmp_path / "libsage.so"))
+    monkeypatch.setattr(sage, "_lib", None)
+    with pytest.raises(ImportError):
+        sage.lib()
+    with pytest.raises(ImportError):
+        sage.sage_attn_workspace_bytes(1, 1, 128, 64)
