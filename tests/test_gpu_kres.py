@@ -28,6 +28,7 @@ CASES = [
     tiny_custom(1, 2, 777, 128, 602, layout="fused", bias_sigma=4.0, outlier_frac=0.01),
     tiny_custom(2, 3, 200, 128, 603, bias_sigma=4.0, outlier_frac=0.02),
     tiny_custom(1, 1, 50, 64, 604),
+    tiny_custom(1, 2, 1, 64, 605, bias_sigma=1.0),
     WORKLOADS["tiny"],
 ]
 

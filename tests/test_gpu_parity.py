@@ -325,6 +325,7 @@ def test_device_error_word_is_clear():
     tiny_custom(1, 2, 300, 64, 701, layout="fused", bias_sigma=2.0),
     tiny_custom(2, 3, 777, 128, 702, bias_sigma=4.0, outlier_frac=0.01),
     tiny_custom(1, 1, 50, 128, 703, layout="fused"),
+    tiny_custom(1, 2, 1, 64, 704),
     WORKLOADS["flux"],
 ], ids=lambda w: w.name)
 def test_prologue_q_quantization_forward_is_bit_identical(w):
