@@ -725,8 +725,13 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         } else if (ok && !EXPORT_S && wait_warp(&ctl->o_final[t], 0, p.err, &ctl->abort, 13)) {
             tc_fence_after();
             const float inv_l = 1.f / l;
-            uint16_t *orow = p.out + (int64_t)(bh / p.H) * p.osb + (int64_t)(bh % p.H) * p.osh +
-                             (int64_t)grow * p.osn;
+            // The warp's 32 bf16 rows go through its share of the tile's P buffers
+            // (free: every P.V has completed) so that the global stores cover
+            // whole rows: 16-byte chunk c of row r is staged at r*2d +
+            // ((c ^ (r mod CPR)) * 16), then each store instruction writes
+            // 32 * 16 bytes = 512 / (2d) rows.
+            constexpr int CPR = D / 8;  // 16-byte chunks per row
+            const uint32_t stage = pbase + (row - lane) * D * 2;  // the warp's 32 rows of its tile's P buffers
 #pragma unroll 1
             for (int cc = 0; cc < D / 32; ++cc) {
                 uint32_t o[32];
@@ -739,12 +744,23 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                     w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * ctl->v_scale[cidx] * inv_l,
                                        __uint_as_float(o[2 * i + 1]) * ctl->v_scale[cidx + 1] * inv_l);
                 }
-                if (grow < p.N) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(orow + cc * 32);
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    const int c = cc * 4 + i;
+                    st_shared_v4(stage + lane * D * 2 + ((c ^ (lane & (CPR - 1))) << 4), w[4 * i], w[4 * i + 1],
+                                 w[4 * i + 2], w[4 * i + 3]);
                 }
+            }
+            __syncwarp();
+            constexpr int RPI = 32 / CPR;  // rows per store instruction
+            const int c = lane % CPR;
+            uint16_t *obase = p.out + (int64_t)(bh / p.H) * p.osb + (int64_t)(bh % p.H) * p.osh;
+#pragma unroll 1
+            for (int r0 = 0; r0 < 32; r0 += RPI) {
+                const int r = r0 + lane / CPR;
+                const uint4 val = ld_shared_v4(stage + r * D * 2 + ((c ^ (r & (CPR - 1))) << 4));
+                const int gr = grow - lane + r;  // this warp's first row is grow - lane
+                if (gr < p.N) *reinterpret_cast<uint4 *>(obase + (int64_t)gr * p.osn + c * 8) = val;
             }
         }
     }
