@@ -50,7 +50,8 @@
 // 64-key block; running max m' = max(m, ceil(rowmax x)) so that the O / l
 // rescale 2^(m-m') is an exact power of two; P = e4m3(2^(x-m') * 448) computed as
 // 2^(x - m' + log2 448); l accumulates the unrounded values; the epilogue
-// writes bf16(O * v_scale / l).
+// writes bf16(O * v_scale / l), staging each warp's rows in its tile's (then
+// idle) P buffers so that every store instruction covers whole output rows.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
