@@ -212,7 +212,7 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint32_t a, uint32_
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(saddr), "r"(a), "r"(b), "r"(c), "r"(d)
                  : "memory");
 }
-// 8-byte shared-memory store.
+// 16-byte shared-memory load.
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
@@ -221,6 +221,7 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t saddr) {
                  : "memory");
     return v;
 }
+// 8-byte shared-memory store.
 __device__ __forceinline__ void st_shared_v2(uint32_t saddr, uint32_t a, uint32_t b) {
     asm volatile("st.shared.v2.b32 [%0], {%1, %2};" ::"r"(saddr), "r"(a), "r"(b) : "memory");
 }
