@@ -327,6 +327,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         tma_prefetch_desc(&tm_k);
         if (!EXPORT_S) tma_prefetch_desc(&tm_v);
     }
+    // everything below reads what the previous kernel of the stream wrote
+    grid_dep_wait();
     for (int i = threadIdx.x; i < D; i += blockDim.x) ctl->v_scale[i] = EXPORT_S ? 0.f : p.v_scale[bh * D + i];
     if constexpr (SPARSE) {
         // a tile past the last query tile keeps nothing
@@ -841,8 +843,7 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
     if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    kern<<<grid, C::THREADS, smem, st>>>(tq, tk, tv, tqb, p);
-    return cudaGetLastError();
+    return launch_dependent(kern, grid, dim3(C::THREADS), smem, st, tq, tk, tv, tqb, p);
 }
 
 }  // namespace

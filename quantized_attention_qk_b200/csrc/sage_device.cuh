@@ -295,6 +295,12 @@ __device__ __forceinline__ uint64_t smem_desc_mnmajor(uint32_t saddr, uint32_t r
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | (1ull << 16) | (sbo << 32) | (1ull << 46) | (layout << 61);
 }
 
+// Programmatic dependent launch (see launch_dependent): wait until the previous
+// kernel of the stream has completed and its writes are visible (returns at
+// once for a kernel launched the plain way); let the next kernel start launching.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Instruction descriptors (kind::i8 and kind::f8f6f4 share the layout):
 // [4,6) D type (1 f32, 2 s32), [7,10) A type, [10,13) B type, [15] A MN-major,
 // [16] B MN-major, [17,23) N>>3, [24,29) M>>4.

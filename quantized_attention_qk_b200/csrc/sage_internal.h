@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace sage {
 
 constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
@@ -82,6 +84,27 @@ cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *
 cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped);
 // Device error word (bounded waits that gave up) of the current device.
 unsigned *device_error_ptr();
+
+// Launch `kern` with programmatic stream serialization: its CTAs may start
+// while the previous kernel of `st` is still running (once every CTA of that
+// kernel has signalled griddepcontrol.launch_dependents or exited).  The kernel
+// executes griddepcontrol.wait before it reads or writes anything an earlier
+// kernel of the stream writes or reads; the first kernel of a forward is
+// launched the plain way, so each forward starts after the previous one ended.
+template <typename... P, typename... A>
+cudaError_t launch_dependent(void (*kern)(P...), dim3 grid, dim3 block, int smem, cudaStream_t st, A &&...args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<A>(args)...);
+}
 
 // Attention launchers (sage_attn.cu).
 cudaError_t launch_attention(const Shape &s, const Codes &c, const Dst &out, float sm_scale, cudaStream_t st);

@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
     const int i0 = blockIdx.x * a.per, i1 = min(n_items, i0 + a.per);
     const int cv = threadIdx.x % VPR, r0 = threadIdx.x / VPR;
     const uint32_t bytes = (a.do_k + a.do_v) * TILE * 2;
+    grid_dep_launch();  // the quantize kernel may take each SM this CTA leaves
     auto rows_of = [&](int item) {
         const int n0 = (item % a.nch) * a.chunk;
         return min(a.N, n0 + a.chunk) - n0;
@@ -270,10 +271,15 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
         if (DO_V) load_rows<D>(base + OV * TILE, kQBlock, &tv, a.v_swap, &bar[buf], blk * kQBlock, h, b, drop);
     };
     int issued = 0, waited = 0;  // thread 0: loads issued, and seen complete
+    grid_dep_launch();  // the attention kernel may take each SM this CTA leaves
+    // The rows are the caller's inputs, complete before the statistics kernel
+    // started: the first item's loads go out before the wait for that kernel's
+    // partials (and before anything here is written).
     if (threadIdx.x == 0 && i0 < i1) {
         issue(i0, 0);
         issued = 1;
     }
+    grid_dep_wait();
     int cur_bh = -1;
     for (int item = i0, k = 0; item < i1; ++item, ++k) {
         const int buf = k & 1;
@@ -477,8 +483,8 @@ cudaError_t launch_quant_k(const Shape &s, const CUtensorMap &tq, const CUtensor
     const int ctas = resident_ctas(kern, quant_threads<D>(), smem);
     if (ctas <= 0) return cudaErrorInvalidConfiguration;
     a.per = (items + ctas - 1) / ctas;
-    kern<<<(items + a.per - 1) / a.per, quant_threads<D>(), smem, st>>>(tq, tk, tv, a);
-    return cudaGetLastError();
+    return launch_dependent(kern, dim3((items + a.per - 1) / a.per), dim3(quant_threads<D>()), smem, st, tq, tk, tv,
+                            a);
 }
 
 template <int D>
