@@ -40,6 +40,13 @@
  *     of 8 elements (16-byte vectors).  Otherwise SAGE_ERR_INVALID_ARG (bad
  *     pointer/stride/shape/scale) or SAGE_ERR_UNSUPPORTED (d, dtype) is
  *     returned before anything is launched.
+ *   - Input values are finite.  With an infinity or NaN in a block the codes of
+ *     that block (and every output that uses them) are unspecified; nothing
+ *     checks for it.
+ *   - A forward launches its kernels back to back on `stream`; all but the
+ *     first may begin while their predecessor finishes (programmatic dependent
+ *     launch) and wait on the device for its results, so the call's ordering
+ *     with respect to other work on `stream` is the ordinary stream order.
  *   - N_pad = ceil(N/128)*128.  Padded rows of every code buffer are written
  *     as zeros; padded blocks get scale 0.
  *   - Every device buffer is owned by the caller; the library keeps no pointer
