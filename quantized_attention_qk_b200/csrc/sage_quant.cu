@@ -63,9 +63,14 @@ __device__ __forceinline__ void load_rows(uint16_t *tile, int rows, const CUtens
 }
 
 // Max over the block of three values at once (all threads get the results).
+// `sh` holds two slot sets [2][3][NT/32], used alternately (`set`): a set is
+// written again only by the call after next, which every thread reaches after
+// the next call's barrier, i.e. after all threads have read this call's slots;
+// so one barrier per call suffices.
 template <int NT>
-__device__ __forceinline__ void block_max3_n(float &a, float &b, float &c, float *sh /*[3][NT/32]*/) {
+__device__ __forceinline__ void block_max3_n(float &a, float &b, float &c, float *shs, int set) {
     constexpr int NW = NT / 32;
+    float *sh = shs + set * 3 * NW;
     a = warp_max(a);
     b = warp_max(b);
     c = warp_max(c);
@@ -77,7 +82,6 @@ __device__ __forceinline__ void block_max3_n(float &a, float &b, float &c, float
     c = sh[2 * NW];
 #pragma unroll
     for (int i = 1; i < NW; ++i) { a = fmaxf(a, sh[i]); b = fmaxf(b, sh[NW + i]); c = fmaxf(c, sh[2 * NW + i]); }
-    __syncthreads();
 }
 
 // Persistent CTAs over the (b,h, token chunk) items, a contiguous range each,
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
     uint16_t *bufs = reinterpret_cast<uint16_t *>(smem_raw);  // [2][NT][TILE]
     __shared__ uint64_t bar[2];
     __shared__ float mu[D], vinv[D], vmax[D];
-    __shared__ float red[3 * (NTH / 32)];
+    __shared__ float red[2 * 3 * (NTH / 32)];
     __shared__ AbortState abort_st;
     __shared__ int bad;
     const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock;
@@ -283,14 +287,11 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
     int cur_bh = -1;
     for (int item = i0, k = 0; item < i1; ++item, ++k) {
         const int buf = k & 1;
-        if (threadIdx.x == 0 && !bad && item + 1 < i1) {
-            issue(item + 1, buf ^ 1);  // that buffer was released at the end of the last item
-            ++issued;
-        }
         const int bh = item / nqb, blk = item % nqb;
         if ((DO_K || DO_V) && bh != cur_bh) {
             // this (b,h)'s statistics from the chunk partials, in chunk order:
             // mean = sum / N (IEEE divide), V factor 448 / amax
+            __syncthreads();  // every thread is done coding with the previous head's
             for (int c = threadIdx.x; c < D; c += NTH) {
                 float sum = 0.f, mx = 0.f;
 #pragma unroll 8
@@ -311,7 +312,13 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
             else
                 bad = 1;
         }
-        __syncthreads();  // the rows and the statistics are ready
+        // the rows and the statistics are ready, and every thread is done with
+        // the previous item, so its buffer takes the next item's rows
+        __syncthreads();
+        if (threadIdx.x == 0 && !bad && item + 1 < i1) {
+            issue(item + 1, buf ^ 1);
+            ++issued;
+        }
         if (blk == 0 && (DO_K || DO_V)) {
             for (int c = threadIdx.x; c < D; c += NTH) {
                 if (DO_K) {
@@ -362,7 +369,7 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
                     if (row < kKBlock) ka0 = fmaxf(ka0, am); else ka1 = fmaxf(ka1, am);
                 }
             }
-            block_max3_n<NTH>(qa, ka0, ka1, red);
+            block_max3_n<NTH>(qa, ka0, ka1, red, k & 1);
         }
 
         if (DO_Q && !bad) {
@@ -402,18 +409,17 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
                 uint32_t w[4];
 #pragma unroll
                 for (int e = 0; e < 8; e += 2) {
+                    float y0, y1;
+                    fmul2(y0, y1, f[e], f[e + 1], inv[e], inv[e + 1]);  // IEEE products; nothing is added
                     uint16_t pr;
                     // cvt packs its first source in the high byte: (hi=e+1, lo=e)
-                    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;"
-                        : "=h"(pr)
-                        : "f"(__fmul_rn(f[e + 1], inv[e + 1])), "f"(__fmul_rn(f[e], inv[e])));
+                    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(y1), "f"(y0));
                     w[e / 2] = pr;
                 }
                 *reinterpret_cast<uint2 *>(dst + (int64_t)(r0 + i * RPI) * D) =
                     make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
             }
         }
-        __syncthreads();  // the buffer and the statistics may be replaced
     }
     if (threadIdx.x == 0) {
         // every copy started here lands before the CTA exits
