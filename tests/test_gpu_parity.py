@@ -284,6 +284,31 @@ def test_repeat_calls_are_deterministic():
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+def test_back_to_back_forwards_sharing_a_workspace_do_not_interfere():
+    """The kernels after the first of a forward may start before their
+    predecessor ends (programmatic dependent launch); the first kernel of a
+    forward may not, so the next forward cannot overwrite the codes the previous
+    forward's attention kernel still reads.  Several forwards of different
+    inputs go out back to back on one stream into one workspace, with no
+    synchronisation between them; each output must equal its own forward run
+    alone, bit for bit."""
+    ws_ = [tiny_custom(1, 24, 4608, 128, seed=70 + i, layout="fused", bias_sigma=2.0) for i in range(3)]
+    ins = [_inputs(w)[1] for w in ws_]
+    alone = []
+    for (qd, kd, vd) in ins:
+        alone.append(sage.sage_attn_fwd(qd, kd, vd))
+        torch.cuda.synchronize()
+    ws = torch.empty(sage.sage_attn_workspace_bytes(1, 24, 4608, 128), dtype=torch.uint8, device=DEV)
+    outs = [torch.empty(1, 24, 4608, 128, dtype=torch.bfloat16, device=DEV) for _ in ins]
+    for rep in range(3):
+        for (qd, kd, vd), o in zip(ins, outs):
+            sage.sage_attn_fwd(qd, kd, vd, out=o, workspace=ws)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    for a, o in zip(alone, outs):
+        assert torch.equal(a.view(torch.int16), o.view(torch.int16))
+
+
 # --------------------------------------------------------------------------- dense reference and exact
 
 @pytest.mark.parametrize("name", ["tiny", "sdxl"])
