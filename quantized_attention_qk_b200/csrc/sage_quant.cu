@@ -19,6 +19,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 #include "sage_device.cuh"
 #include "sage_internal.h"
 
@@ -427,6 +429,21 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
     }
 }
 
+// Raise a kernel's dynamic shared-memory limit on the current device once:
+// the attribute belongs to the device, so `done` keeps one bit per device
+// index (indices past 63 set it on every call).
+template <typename K>
+cudaError_t ensure_smem_limit(K kern, int smem, std::atomic<uint64_t> &done) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
+    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
+    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
+    done.fetch_or(bit, std::memory_order_relaxed);
+    return cudaSuccess;
+}
+
 // CTAs that fit at once on the device for a kernel and its dynamic shared memory.
 template <typename K>
 int resident_ctas(K kern, int threads, int smem) {
@@ -458,12 +475,8 @@ cudaError_t launch_stats_d(const Shape &s, const Src *k, const Src *v, const Sta
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
     constexpr int RPI = kThreads / (D / 8);
     const int smem = kStatsStages * 2 * kRowsPerLoad * D * 2 + 2 * RPI * D * 4;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[D == 128]) {
-        if ((e = cudaFuncSetAttribute(k_stats<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-            return e;
-        attr_set[D == 128] = true;
-    }
+    static std::atomic<uint64_t> limit_set{0};  // one per instantiation
+    if ((e = ensure_smem_limit(k_stats<D>, smem, limit_set)) != cudaSuccess) return e;
     const int items = a.nch * s.BH();
     const int ctas = resident_ctas(k_stats<D>, kThreads, smem);
     if (ctas <= 0) return cudaErrorInvalidConfiguration;
@@ -478,13 +491,9 @@ cudaError_t launch_quant_k(const Shape &s, const CUtensorMap &tq, const CUtensor
     constexpr int NT = (DQ ? 1 : 0) + (DK ? 1 : 0) + (DV ? 1 : 0);
     const int smem = 2 * NT * kQBlock * D * 2;
     auto kern = k_quant<D, DQ, DK, DV>;
-    static bool attr_set = false;  // one per instantiation
+    static std::atomic<uint64_t> limit_set{0};  // one per instantiation
     cudaError_t e;
-    if (!attr_set) {
-        if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess)
-            return e;
-        attr_set = true;
-    }
+    if ((e = ensure_smem_limit(kern, smem, limit_set)) != cudaSuccess) return e;
     const int items = s.n_qblocks() * s.BH();
     const int ctas = resident_ctas(kern, quant_threads<D>(), smem);
     if (ctas <= 0) return cudaErrorInvalidConfiguration;
