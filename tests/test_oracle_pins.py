@@ -302,3 +302,23 @@ def test_kres_block_mean_term_varies_by_block():
     o, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows, fp8_p=False, fp8_v=False, round_bf16=False,
                              k_residual=True)
     assert np.linalg.norm(o - ex) / np.linalg.norm(ex) < 0.03
+
+
+def test_kres_constant_block_has_zero_residual():
+    """A K block whose rows are all equal is its own mean: the residual codes and
+    the block scale are 0, and with the remaining rounding switched off the
+    scores of that block are the mean term alone, so attention is exact."""
+    w = tiny_custom(1, 1, 128, 64, seed=94, bias_sigma=1.0)
+    q, k, v, _ = make_qkv(w)
+    k = k.clone()
+    k[0, 0, :64] = k[0, 0, 5]            # block 0: one repeated bf16 row
+    got = oracle.quantize_kres(k)
+    assert np.all(got["k_i8"][0, 0, :64] == 0)
+    assert got["k_scale"][0, 0, 0] == 0.0
+    mb = torch.from_numpy(got["k_bmean"][0, 0, 0].astype(np.int16)).view(torch.bfloat16)
+    assert torch.equal(mb, k[0, 0, 5])   # the mean of equal bf16 values is that value
+    rows = np.arange(0, 128, 3).astype(np.int32)
+    ex = oracle.attn_exact(q, k, v, w.sm_scale, rows=rows)
+    o, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows, int8_qk=False, fp8_p=False, fp8_v=False,
+                             round_bf16=False, k_residual=True)
+    assert np.max(np.abs(o - ex)) < 1e-12
