@@ -322,3 +322,67 @@ def test_kres_constant_block_has_zero_residual():
     o, _ = oracle.attn_quant(q, k, v, w.sm_scale, rows=rows, int8_qk=False, fp8_p=False, fp8_v=False,
                              round_bf16=False, k_residual=True)
     assert np.max(np.abs(o - ex)) < 1e-12
+
+
+# --------------------------------------------------------------------------
+# integer score tiles (the closed form the GPU's S tiles are checked against)
+# --------------------------------------------------------------------------
+
+def _int8_codes(shape, rng):
+    return rng.integers(-127, 128, size=shape).astype(np.int8)
+
+
+@pytest.mark.parametrize("m,n,d", [(1, 1, 1), (3, 5, 64), (7, 2, 128), (5, 9, 33)])
+def test_int8_gemm_nt_equals_python_integer_loops(m, n, d):
+    """s[i][j] = sum_c a[i][c] b[j][c] over Python ints, with rows at +-127."""
+    rng = np.random.default_rng(1000 * m + 10 * n + d)
+    a, b = _int8_codes((m, d), rng), _int8_codes((n, d), rng)
+    a[0] = -127                       # extreme rows: |s| = 127 * 127 * d
+    b[-1] = -127
+    got = oracle.int8_gemm_nt(a, b)
+    assert got.shape == (m, n) and got.dtype == np.int32
+    for i in range(m):
+        for j in range(n):
+            want = sum(int(a[i, c]) * int(b[j, c]) for c in range(d))
+            assert int(got[i, j]) == want, (i, j)
+    assert int(got[0, n - 1]) == 127 * 127 * d
+
+
+@pytest.mark.parametrize("m,n,d", [(128, 96, 128), (40, 128, 64), (128, 128, 128)])
+def test_int8_gemm_nt_equals_int64_product_not_transposed(m, n, d):
+    """Against the int64 matrix product a b^T (m != n catches a swapped
+    operand or a transposed result), including the largest magnitudes."""
+    rng = np.random.default_rng(7 * m + n + d)
+    a, b = _int8_codes((m, d), rng), _int8_codes((n, d), rng)
+    a[1] = 127
+    a[2] = -127
+    b[3] = -127
+    got = oracle.int8_gemm_nt(a, b)
+    want = a.astype(np.int64) @ b.astype(np.int64).T
+    np.testing.assert_array_equal(got.astype(np.int64), want)
+    assert got[2, 3] == 127 * 127 * d and got[1, 3] == -127 * 127 * d
+
+
+def test_int8_gemm_nt_indexes_rows_and_channels():
+    """One nonzero code per row: s[i][j] is nonzero only where a's channel of
+    row i meets b's channel of row j, so a swapped index shows at once; the
+    row strides of the C routine are exercised with padded rows."""
+    m, n, d, pad = 6, 4, 16, 24
+    a = np.zeros((m, pad), np.int8)
+    b = np.zeros((n, pad), np.int8)
+    ca = [0, 3, 5, 7, 9, 15]
+    cb = [3, 9, 0, 15]
+    for i, c in enumerate(ca):
+        a[i, c] = i + 1
+        a[i, d:] = 99                 # padding past d must not be read
+    for j, c in enumerate(cb):
+        b[j, c] = -(j + 2)
+        b[j, d:] = 99
+    s = np.zeros((m, n), np.int32)
+    L = oracle.lib()
+    rc = L.oracle_int8_gemm_nt(oracle._ptr(a), pad, oracle._ptr(b), pad, m, n, d, oracle._ptr(s))
+    assert rc == 0
+    for i in range(m):
+        for j in range(n):
+            want = (i + 1) * -(j + 2) if ca[i] == cb[j] else 0
+            assert s[i, j] == want, (i, j)
