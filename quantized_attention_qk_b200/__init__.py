@@ -99,6 +99,14 @@ def _raise(status: int):
         raise SageError(status, lib().sage_last_error_message().decode(errors="replace"))
 
 
+def _run(dev, fn, *args):
+    """Call library function ``fn`` with ``dev`` as the current device: the
+    library launches its kernels on, and keeps its per-device state for, the
+    current device, and rejects tensors that live elsewhere."""
+    with torch.cuda.device(dev):
+        _raise(fn(*args))
+
+
 def _strides(t: torch.Tensor):
     return (ctypes.c_int64 * 4)(*t.stride())
 
@@ -131,7 +139,8 @@ def sage_quant_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
 
 
 def sage_check(stream=None, device=None):
-    _raise(lib().sage_check(_stream(stream, device)))
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    _run(dev, lib().sage_check, _stream(stream, dev))
 
 
 def sage_quant_qk(q, k, workspace=None, stream=None):
@@ -147,9 +156,9 @@ def sage_quant_qk(q, k, workspace=None, stream=None):
              k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
              k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev))
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _raise(lib().sage_quant_qk(_ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
+    _run(dev, lib().sage_quant_qk, _ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
                                _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]), _ptr(r["k_scale"]),
-                               _ptr(r["k_mean"]), _ptr(workspace), ws_bytes, _stream(stream, dev)))
+                               _ptr(r["k_mean"]), _ptr(workspace), ws_bytes, _stream(stream, dev))
     return r
 
 
@@ -157,7 +166,7 @@ def sage_quant_qk_noalloc(q, k, out=None, stream=None):
     """sage_quant_qk without a workspace and without any device allocation in
     the library: its statistics scratch is a fixed 4 MiB array in the library's
     device memory (shared by all calls on a device; calls that overlap on the
-    GPU race).  ``out`` optionally supplies the output dict (same keys/shapes as
+    GPU race; shapes needing more scratch raise with status 3).  ``out`` optionally supplies the output dict (same keys/shapes as
     sage_quant_qk returns) so that the caller owns every buffer."""
     _check_qkv(q, k)
     B, H, N, d = q.shape
@@ -169,9 +178,9 @@ def sage_quant_qk_noalloc(q, k, out=None, stream=None):
         k_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
         k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
         k_mean=torch.empty(B, H, d, dtype=torch.float32, device=dev))
-    _raise(lib().sage_quant_qk_noalloc(_ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
+    _run(dev, lib().sage_quant_qk_noalloc, _ptr(q), _strides(q), _ptr(k), _strides(k), B, H, N, d,
                                        _ptr(r["q_i8"]), _ptr(r["q_scale"]), _ptr(r["k_i8"]), _ptr(r["k_scale"]),
-                                       _ptr(r["k_mean"]), _stream(stream, dev)))
+                                       _ptr(r["k_mean"]), _stream(stream, dev))
     return r
 
 
@@ -183,8 +192,8 @@ def sage_quant_v(v, workspace=None, stream=None):
     v_e4m3 = torch.empty(B, H, n_pad(N), d, dtype=torch.uint8, device=dev)
     v_scale = torch.empty(B, H, d, dtype=torch.float32, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _raise(lib().sage_quant_v(_ptr(v), _strides(v), B, H, N, d, _ptr(v_e4m3), _ptr(v_scale), _ptr(workspace),
-                              ws_bytes, _stream(stream, dev)))
+    _run(dev, lib().sage_quant_v, _ptr(v), _strides(v), B, H, N, d, _ptr(v_e4m3), _ptr(v_scale), _ptr(workspace),
+                              ws_bytes, _stream(stream, dev))
     return v_e4m3, v_scale
 
 
@@ -199,9 +208,9 @@ def sage_attn_quantized(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, N: int, s
     for t in (q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale):
         if not t.is_contiguous():
             raise ValueError("code and scale tensors must be contiguous")
-    _raise(lib().sage_attn_quantized(_ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_e4m3),
+    _run(dev, lib().sage_attn_quantized, _ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale), _ptr(v_e4m3),
                                      _ptr(v_scale), _ptr(out), _strides(out), B, H, N, d,
-                                     ctypes.c_float(sm_scale), _stream(stream, dev)))
+                                     ctypes.c_float(sm_scale), _stream(stream, dev))
     return out
 
 
@@ -218,14 +227,14 @@ def sage_attn_fwd(q, k, v, sm_scale=None, out=None, workspace=None, stream=None,
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     if attn_events is None:
-        _raise(lib().sage_attn_fwd(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+        _run(dev, lib().sage_attn_fwd, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                    _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                                   _ptr(workspace), ws_bytes, _stream(stream, dev)))
+                                   _ptr(workspace), ws_bytes, _stream(stream, dev))
     else:
         e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events)
-        _raise(lib().sage_attn_fwd_ev(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+        _run(dev, lib().sage_attn_fwd_ev, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                       _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                                      _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
+                                      _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1)
     return out
 
 
@@ -237,9 +246,9 @@ def sage_attn_dense_ref_gpu(q, k, v, sm_scale=None, out=None, stream=None):
         sm_scale = 1.0 / math.sqrt(d)
     if out is None:
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=q.device)
-    _raise(lib().sage_attn_dense_ref_gpu(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+    _run(q.device, lib().sage_attn_dense_ref_gpu, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                          _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                                         _stream(stream, q.device)))
+                                         _stream(stream, q.device))
     return out
 
 
@@ -247,8 +256,8 @@ def sage_debug_qk_tile(q_i8, k_i8, N: int, b: int, h: int, q_tile: int, kv_tile:
     """int32 [128,128] S tile of slab (b,h) computed on the tcgen05 INT8 path."""
     B, H, _, d = q_i8.shape
     s = torch.empty(128, 128, dtype=torch.int32, device=q_i8.device)
-    _raise(lib().sage_debug_qk_tile(_ptr(q_i8), _ptr(k_i8), B, H, N, d, b, h, q_tile, kv_tile, _ptr(s),
-                                    _stream(stream, q_i8.device)))
+    _run(q_i8.device, lib().sage_debug_qk_tile, _ptr(q_i8), _ptr(k_i8), B, H, N, d, b, h, q_tile, kv_tile, _ptr(s),
+                                    _stream(stream, q_i8.device))
     return s
 
 
@@ -351,9 +360,9 @@ def sage_block_select(codes, N: int, sm_scale: float, tau: float, want_scores=Fa
     mask = torch.empty(B, H, T, W, dtype=torch.int32, device=dev)
     scores = torch.empty(B, H, T, T, dtype=torch.float32, device=dev) if want_scores else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _raise(lib().sage_block_select(_ptr(q_i8), _ptr(codes["q_scale"]), _ptr(k_i8), _ptr(codes["k_scale"]),
+    _run(dev, lib().sage_block_select, _ptr(q_i8), _ptr(codes["q_scale"]), _ptr(k_i8), _ptr(codes["k_scale"]),
                                    B, H, N, d, ctypes.c_float(sm_scale), ctypes.c_float(tau), _ptr(mask),
-                                   _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream, dev)))
+                                   _ptr(scores), _ptr(workspace), ws_bytes, _stream(stream, dev))
     return (mask, scores) if want_scores else mask
 
 
@@ -375,10 +384,10 @@ def sage_attn_fwd_sparse(q, k, v, tau=1.0, sm_scale=None, mask=None, return_mask
         mask_out = torch.empty(B, H, n_tiles(N), mask_words(N), dtype=torch.int32, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
-    _raise(lib().sage_attn_fwd_sparse(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+    _run(dev, lib().sage_attn_fwd_sparse, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                       _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
                                       ctypes.c_float(tau), _ptr(mask), _ptr(mask_out), _ptr(workspace), ws_bytes,
-                                      _stream(stream, dev), e0, e1))
+                                      _stream(stream, dev), e0, e1)
     return (out, mask_out) if return_mask else out
 
 
@@ -400,8 +409,8 @@ def sage_quant_k_residual(k, stream=None):
     r = dict(k_i8=torch.empty(B, H, npd, d, dtype=torch.int8, device=dev),
              k_scale=torch.empty(B, H, npd // K_BLOCK, dtype=torch.float32, device=dev),
              k_bmean=torch.empty(B, H, npd // K_BLOCK, d, dtype=torch.int16, device=dev))
-    _raise(lib().sage_quant_k_residual(_ptr(k), _strides(k), B, H, N, d, _ptr(r["k_i8"]), _ptr(r["k_scale"]),
-                                       _ptr(r["k_bmean"]), _stream(stream, dev)))
+    _run(dev, lib().sage_quant_k_residual, _ptr(k), _strides(k), B, H, N, d, _ptr(r["k_i8"]), _ptr(r["k_scale"]),
+                                       _ptr(r["k_bmean"]), _stream(stream, dev))
     return r
 
 
@@ -416,9 +425,9 @@ def sage_attn_fwd_kres(q, k, v, sm_scale=None, out=None, workspace=None, stream=
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
-    _raise(lib().sage_attn_fwd_kres(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+    _run(dev, lib().sage_attn_fwd_kres, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                     _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                                    _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
+                                    _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1)
     return out
 
 
@@ -434,9 +443,9 @@ def sage_attn_fwd_fused_q(q, k, v, sm_scale=None, out=None, workspace=None, stre
         out = torch.empty(B, H, N, d, dtype=torch.bfloat16, device=dev)
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     e0, e1 = (ctypes.c_void_p(e.cuda_event) for e in attn_events) if attn_events is not None else (None, None)
-    _raise(lib().sage_attn_fwd_fused_q(_ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
+    _run(dev, lib().sage_attn_fwd_fused_q, _ptr(q), _strides(q), _ptr(k), _strides(k), _ptr(v), _strides(v),
                                        _ptr(out), _strides(out), B, H, N, d, ctypes.c_float(sm_scale),
-                                       _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1))
+                                       _ptr(workspace), ws_bytes, _stream(stream, dev), e0, e1)
     return out
 
 
@@ -444,4 +453,4 @@ def sage_debug_wait_timeout(microseconds: int = 10000, stream=None, device=None)
     """Launch the bounded-wait probe (include/sage.h): the next sage_check on
     the stream reports SAGE_ERR_TIMEOUT."""
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
-    _raise(lib().sage_debug_wait_timeout(int(microseconds), _stream(stream, dev)))
+    _run(dev, lib().sage_debug_wait_timeout, int(microseconds), _stream(stream, dev))

@@ -36,14 +36,6 @@ sage_status_t cuda_fail(cudaError_t e, const char *what) {
 constexpr size_t kAlign = 1024;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-sage_status_t check_shape(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1) return fail(SAGE_ERR_INVALID_ARG, "shape B=%d H=%d N=%d must be positive", B, H, N);
-    if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d=%d is not supported (64 or 128)", d);
-    if ((int64_t)B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
-    if (N > (1 << 24)) return fail(SAGE_ERR_UNSUPPORTED, "N=%d exceeds 2^24 tokens", N);
-    return SAGE_OK;
-}
-
 // bf16 tensor view: 16-byte aligned base, channel stride 1, other strides
 // multiples of 8 elements (so every row starts on a 16-byte boundary).
 sage_status_t check_view(const void *p, const int64_t *st, const char *name) {
@@ -95,6 +87,30 @@ sage_status_t get_scratch(Scratch &s, void *ws, size_t ws_bytes, size_t need, cu
 
 }  // namespace
 
+sage_status_t check_shape(int B, int H, int N, int d) {
+    if (B < 1 || H < 1 || N < 1) return fail(SAGE_ERR_INVALID_ARG, "shape B=%d H=%d N=%d must be positive", B, H, N);
+    if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d=%d is not supported (64 or 128)", d);
+    if ((int64_t)B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
+    if (N > (1 << 24)) return fail(SAGE_ERR_UNSUPPORTED, "N=%d exceeds 2^24 tokens", N);
+    return SAGE_OK;
+}
+
+sage_status_t check_on_current_device(const void *p, const char *name) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    cudaPointerAttributes a{};
+    if ((e = cudaPointerGetAttributes(&a, p)) != cudaSuccess) {
+        cudaGetLastError();  // the query's error is not sticky; clear it
+        return fail(SAGE_ERR_INVALID_ARG, "%s: %s", name, cudaGetErrorString(e));
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+        return fail(SAGE_ERR_INVALID_ARG, "%s is not device memory", name);
+    if (a.device != dev)
+        return fail(SAGE_ERR_INVALID_ARG, "%s is on device %d but device %d is current", name, a.device, dev);
+    return SAGE_OK;
+}
+
 void set_last_error(const char *fmt, ...) {
     char buf[512];
     va_list ap;
@@ -104,21 +120,24 @@ void set_last_error(const char *fmt, ...) {
     g_last_error = buf;
 }
 
+// Statistics scratch: fp64 K column sums and fp32 V column maxima per
+// 256-token chunk, then the fp32 K mean and V factor per (b,h, channel).
 size_t stats_ws_bytes(const Shape &s) {
-    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d * sizeof(float);
+    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d;
     const size_t per = (size_t)s.BH() * s.d * sizeof(float);
-    return 2 * up(part) + 2 * up(per);
+    return up(part * sizeof(double)) + up(part * sizeof(float)) + 2 * up(per);
 }
 
 StatsWs carve_stats_ws(void *base, const Shape &s) {
     char *p = static_cast<char *>(base);
-    const size_t part = up((size_t)s.BH() * s.n_chunks() * s.d * sizeof(float));
+    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d;
+    const size_t kpart = up(part * sizeof(double)), vpart = up(part * sizeof(float));
     const size_t per = up((size_t)s.BH() * s.d * sizeof(float));
     StatsWs w;
-    w.ksum_part = reinterpret_cast<float *>(p);
-    w.vmax_part = reinterpret_cast<float *>(p + part);
-    w.k_mean = reinterpret_cast<float *>(p + 2 * part);
-    w.v_inv = reinterpret_cast<float *>(p + 2 * part + per);
+    w.ksum_part = reinterpret_cast<double *>(p);
+    w.vmax_part = reinterpret_cast<float *>(p + kpart);
+    w.k_mean = reinterpret_cast<float *>(p + kpart + vpart);
+    w.v_inv = reinterpret_cast<float *>(p + kpart + vpart + per);
     return w;
 }
 
@@ -193,7 +212,8 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4], const
     if ((r = check_shape(B, H, N, d)) || (r = check_view(q_bf16, q_stride, "q")) ||
         (r = check_view(k_bf16, k_stride, "k")) || (r = check_dev(q_i8, "q_i8", 16)) ||
         (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(q_scale, "q_scale", 4)) ||
-        (r = check_dev(k_scale, "k_scale", 4)))
+        (r = check_dev(k_scale, "k_scale", 4)) || (r = check_on_current_device(q_bf16, "q")) ||
+        (r = check_on_current_device(q_i8, "q_i8")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -217,7 +237,8 @@ sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B,
                            sage_stream_t stream) {
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_view(v_bf16, v_stride, "v")) ||
-        (r = check_dev(v_e4m3, "v_e4m3", 16)) || (r = check_dev(v_scale, "v_scale", 4)))
+        (r = check_dev(v_e4m3, "v_e4m3", 16)) || (r = check_dev(v_scale, "v_scale", 4)) ||
+        (r = check_on_current_device(v_bf16, "v")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -247,7 +268,8 @@ sage_status_t sage_attn_quantized(const int8_t *q_i8, const float *q_scale, cons
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_dev(q_i8, "q_i8", 16)) ||
         (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(v_e4m3, "v_e4m3", 16)) ||
         (r = check_dev(q_scale, "q_scale", 4)) || (r = check_dev(k_scale, "k_scale", 4)) ||
-        (r = check_dev(v_scale, "v_scale", 4)) || (r = check_view(out, o_stride, "out")))
+        (r = check_dev(v_scale, "v_scale", 4)) || (r = check_view(out, o_stride, "out")) ||
+        (r = check_on_current_device(q_i8, "q_i8")) || (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     Codes c;
@@ -269,7 +291,8 @@ sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4], const v
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
-        (r = check_view(out, o_stride, "out")))
+        (r = check_view(out, o_stride, "out")) || (r = check_on_current_device(q, "q")) ||
+        (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -336,7 +359,8 @@ sage_status_t sage_block_select(const int8_t *q_i8, const float *q_scale, const 
     if ((r = check_sparse_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_tau(tau)) ||
         (r = check_dev(q_i8, "q_i8", 16)) || (r = check_dev(k_i8, "k_i8", 16)) ||
         (r = check_dev(q_scale, "q_scale", 4)) || (r = check_dev(k_scale, "k_scale", 4)) ||
-        (r = check_dev(mask, "mask", 4)) || (scores && (r = check_dev(scores, "scores", 4))))
+        (r = check_dev(mask, "mask", 4)) || (scores && (r = check_dev(scores, "scores", 4))) ||
+        (r = check_on_current_device(q_i8, "q_i8")) || (r = check_on_current_device(mask, "mask")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -363,7 +387,8 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], con
     if ((r = check_sparse_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
         (r = check_view(out, o_stride, "out")) || (!mask_in && (r = check_tau(tau))) ||
-        (mask_in && (r = check_dev(mask_in, "mask_in", 4))) || (mask_out && (r = check_dev(mask_out, "mask_out", 4))))
+        (mask_in && (r = check_dev(mask_in, "mask_in", 4))) || (mask_out && (r = check_dev(mask_out, "mask_out", 4))) ||
+        (r = check_on_current_device(q, "q")) || (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -409,7 +434,8 @@ sage_status_t sage_attn_fwd_fused_q(const void *q, const int64_t q_stride[4], co
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
-        (r = check_view(out, o_stride, "out")))
+        (r = check_view(out, o_stride, "out")) || (r = check_on_current_device(q, "q")) ||
+        (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -445,7 +471,8 @@ sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_view(k_bf16, k_stride, "k")) ||
         (r = check_dev(k_i8, "k_i8", 16)) || (r = check_dev(k_scale, "k_scale", 4)) ||
-        (r = check_dev(k_bmean, "k_bmean", 16)))
+        (r = check_dev(k_bmean, "k_bmean", 16)) || (r = check_on_current_device(k_bf16, "k")) ||
+        (r = check_on_current_device(k_i8, "k_i8")))
         return r;
     const Shape s{B, H, N, d};
     cudaError_t e = launch_kres(s, src(k_bf16, k_stride), k_i8, k_scale, k_bmean, reinterpret_cast<cudaStream_t>(stream));
@@ -460,7 +487,8 @@ sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4], const
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
-        (r = check_view(out, o_stride, "out")))
+        (r = check_view(out, o_stride, "out")) || (r = check_on_current_device(q, "q")) ||
+        (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -495,7 +523,8 @@ sage_status_t sage_attn_dense_ref_gpu(const void *q, const int64_t q_stride[4], 
     sage_status_t r;
     if ((r = check_shape(B, H, N, d)) || (r = check_scale(sm_scale)) || (r = check_view(q, q_stride, "q")) ||
         (r = check_view(k, k_stride, "k")) || (r = check_view(v, v_stride, "v")) ||
-        (r = check_view(out, o_stride, "out")))
+        (r = check_view(out, o_stride, "out")) || (r = check_on_current_device(q, "q")) ||
+        (r = check_on_current_device(out, "out")))
         return r;
     const Shape s{B, H, N, d};
     cudaError_t e = launch_dense_ref(s, src(q, q_stride), src(k, k_stride), src(v, v_stride), dst(out, o_stride),
@@ -515,6 +544,7 @@ sage_status_t sage_debug_qk_tile(const int8_t *q_i8, const int8_t *k_i8, int B, 
         kv_tile >= s.n_qblocks())
         return fail(SAGE_ERR_INVALID_ARG, "tile (b=%d h=%d q_tile=%d kv_tile=%d) outside the tensor", b, h, q_tile,
                     kv_tile);
+    if ((r = check_on_current_device(q_i8, "q_i8")) || (r = check_on_current_device(s_out, "s_out"))) return r;
     cudaError_t e = launch_debug_qk_tile(s, q_i8, k_i8, b * H + h, q_tile, kv_tile, s_out,
                                          reinterpret_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "debug S tile");

@@ -9,6 +9,8 @@
 
 #include <utility>
 
+#include "sage.h"
+
 namespace sage {
 
 constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
@@ -47,8 +49,11 @@ struct Shape {
 };
 
 // Scratch of the quantize pass: per-chunk partials and the finished statistics.
+// The K column sums are fp64: a sum of bf16 values is exact there whenever the
+// column's values span fewer than 53 bits (every workload here), so the mean
+// does not depend on the order of the additions.
 struct StatsWs {
-    float *ksum_part;  // [BH][chunks][d]
+    double *ksum_part;  // [BH][chunks][d]
     float *vmax_part;  // [BH][chunks][d]
     float *k_mean;     // [BH][d]
     float *v_inv;      // [BH][d]  448 / amax (0 for an all-zero channel)
@@ -66,6 +71,13 @@ struct Codes {
 
 // Record the calling thread's error message (what sage_last_error_message returns).
 void set_last_error(const char *fmt, ...);
+
+// Argument checks shared by the entry points (each records the message):
+// the shape limits every kernel assumes, and that `p` is device memory of the
+// current device (kernels launch on the current device; a pointer of another
+// device would be read across the interconnect or fault).
+sage_status_t check_shape(int B, int H, int N, int d);
+sage_status_t check_on_current_device(const void *p, const char *name);
 
 size_t stats_ws_bytes(const Shape &s);
 StatsWs carve_stats_ws(void *base, const Shape &s);

@@ -11,7 +11,9 @@
 // device share it: calls that overlap on the GPU (e.g. on two streams without
 // ordering between them) race on it and must be serialized by the caller.
 // It keeps the last call's contents; every entry a call reads is written
-// earlier in the same call, so nothing has to start at zero.
+// earlier in the same call, so nothing has to start at zero.  Its device
+// address is looked up once per device and kept: a process that calls
+// cudaDeviceReset and goes on using the library is not supported.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -56,9 +58,8 @@ extern "C" sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t
                                                float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
                                                sage_stream_t stream) {
     using namespace sage;
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128))  // reported by the shape check, before any allocation
-        return sage_quant_qk(q_bf16, q_stride, k_bf16, k_stride, B, H, N, d, q_i8, q_scale, k_i8, k_scale,
-                             k_mean, nullptr, 0, stream);
+    sage_status_t r = check_shape(B, H, N, d);  // before the size arithmetic below
+    if (r != SAGE_OK) return r;
     const Shape s{B, H, N, d};
     const size_t need = stats_ws_bytes(s);
     if (need > kNoAllocScratchBytes) {
@@ -67,6 +68,10 @@ extern "C" sage_status_t sage_quant_qk_noalloc(const void *q_bf16, const int64_t
                        need, kNoAllocScratchBytes);
         return SAGE_ERR_WORKSPACE;
     }
+    // The array below belongs to the current device: the inputs must live there
+    // too, or the kernels (launched on the current device) would write another
+    // device's array.
+    if (q_bf16 && (r = check_on_current_device(q_bf16, "q")) != SAGE_OK) return r;
     void *scratch = nullptr;
     cudaError_t e = scratch_for_current_device(&scratch);
     if (e != cudaSuccess) {

@@ -1,8 +1,9 @@
 // sage_quant.cu -- the quantize pass of the quantized attention forward.
 //
 // Two HBM-bound streaming kernels (no tensor cores: there is no contraction):
-//   k_stats  per (b,h, token chunk): sum of K and max |V| per channel over the
-//            chunk, 64-token blocks staged through a 3-deep TMA ring
+//   k_stats  per (b,h, token chunk): sum of K (fp64, exact for bf16 inputs
+//            whose values span fewer than 53 bits) and max |V| per channel
+//            over the chunk, 64-token blocks staged through a 3-deep TMA ring
 //   k_quant  per (b,h, 128-token block): finishes this (b,h)'s statistics from
 //            the chunk partials (the K mean, the smoothing statistic, and the
 //            448/amax factors of V) while TMA brings the block's Q, K and V
@@ -91,7 +92,8 @@ __device__ __forceinline__ void block_max3_n(float &a, float &b, float &c, float
 struct StatsArgs {
     int H, BH, N, nch, chunk, per;  // per: items per CTA
     int do_k, do_v, k_swap, v_swap;
-    float *ksum_part, *vmax_part;  // [BH][nch][D]
+    double *ksum_part;  // [BH][nch][D]
+    float *vmax_part;   // [BH][nch][D]
     unsigned *err;
 };
 
@@ -103,8 +105,8 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
     constexpr int TILE = kRowsPerLoad * D;  // elements of one tensor in one stage
     extern __shared__ __align__(128) uint8_t smem_raw[];
     uint16_t *ring = reinterpret_cast<uint16_t *>(smem_raw);                    // [stage][K,V][TILE]
-    float *red_s = reinterpret_cast<float *>(ring + kStatsStages * 2 * TILE);  // [RPI][D]
-    float *red_m = red_s + RPI * D;
+    double *red_s = reinterpret_cast<double *>(ring + kStatsStages * 2 * TILE);  // [warps][D]
+    float *red_m = reinterpret_cast<float *>(red_s + (kThreads / 32) * D);      // [RPI][D]
     __shared__ uint64_t full[kStatsStages];
     __shared__ AbortState abort_st;
     __shared__ int bad;
@@ -151,9 +153,10 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
     for (int item = i0; item < i1; ++item) {
         const int rows = rows_of(item);
         const int nsub = (rows + kRowsPerLoad - 1) / kRowsPerLoad;
-        float s[8], m[8];
+        double s[8];
+        float m[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) { s[e] = 0.f; m[e] = 0.f; }
+        for (int e = 0; e < 8; ++e) { s[e] = 0.0; m[e] = 0.f; }
         for (int sb = 0; sb < nsub; ++sb) {
             const int q = qbase + sb;
             const int st = q % kStatsStages;
@@ -174,7 +177,7 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
                         if (a.do_k) {
                             unpack8(ld_tile(kt, tile_off(kRowsPerLoad, row, cv)), f);
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) s[e] += f[e];
+                            for (int e = 0; e < 8; ++e) s[e] = __dadd_rn(s[e], static_cast<double>(f[e]));
                         }
                         if (a.do_v) {
                             unpack8(ld_tile(vt, tile_off(kRowsPerLoad, row, cv)), f);
@@ -191,19 +194,25 @@ __global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUte
             }
         }
         qbase += nsub;
-        // the item's partials: rows of the block in order, then per channel
+        // the item's partials: the K sums of a warp's rows by shuffles (the
+        // lanes VPR apart hold the same channels), then the warps in order;
+        // the V maxima per row of the block, then per channel
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-            red_s[r0 * D + cv * 8 + e] = s[e];
+#pragma unroll
+            for (int o = VPR; o < 32; o <<= 1) s[e] = __dadd_rn(s[e], __shfl_xor_sync(0xffffffffu, s[e], o));
             red_m[r0 * D + cv * 8 + e] = m[e];
+        }
+        if ((threadIdx.x & 31) < VPR) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) red_s[(threadIdx.x >> 5) * D + cv * 8 + e] = s[e];
         }
         __syncthreads();
         for (int c = threadIdx.x; c < D; c += kThreads) {
-            float ss = 0.f, mm = 0.f;
-            for (int r = 0; r < RPI; ++r) {
-                ss += red_s[r * D + c];
-                mm = fmaxf(mm, red_m[r * D + c]);
-            }
+            double ss = 0.0;
+            float mm = 0.f;
+            for (int w = 0; w < kThreads / 32; ++w) ss = __dadd_rn(ss, red_s[w * D + c]);
+            for (int r = 0; r < RPI; ++r) mm = fmaxf(mm, red_m[r * D + c]);
             const int64_t o = (int64_t)item * D + c;  // item = bh * nch + chunk
             if (a.do_k) a.ksum_part[o] = ss;
             if (a.do_v) a.vmax_part[o] = mm;
@@ -228,7 +237,8 @@ __host__ __device__ constexpr int quant_threads() { return D == 128 ? 512 : 256;
 struct QuantArgs {
     int H, BH, N, n_pad, nch, per;
     int q_swap, k_swap, v_swap;
-    const float *ksum_part, *vmax_part;  // [BH][nch][D]
+    const double *ksum_part;  // [BH][nch][D]
+    const float *vmax_part;   // [BH][nch][D]
     float *ws_k_mean, *ws_v_inv;         // [BH][D], written with the first block of each (b,h)
     float *user_k_mean;                  // optional copy of the K mean
     Codes c;
@@ -292,17 +302,19 @@ __global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) 
         const int bh = item / nqb, blk = item % nqb;
         if ((DO_K || DO_V) && bh != cur_bh) {
             // this (b,h)'s statistics from the chunk partials, in chunk order:
-            // mean = sum / N (IEEE divide), V factor 448 / amax
+            // mean = fp32(fp64 sum / N) (IEEE divide, then one rounding to
+            // fp32), V factor 448 / amax
             __syncthreads();  // every thread is done coding with the previous head's
             for (int c = threadIdx.x; c < D; c += NTH) {
-                float sum = 0.f, mx = 0.f;
+                double sum = 0.0;
+                float mx = 0.f;
 #pragma unroll 8
                 for (int ch = 0; ch < a.nch; ++ch) {
                     const int64_t o = ((int64_t)bh * a.nch + ch) * D + c;
-                    if (DO_K) sum += a.ksum_part[o];
+                    if (DO_K) sum = __dadd_rn(sum, a.ksum_part[o]);
                     if (DO_V) mx = fmaxf(mx, a.vmax_part[o]);
                 }
-                mu[c] = sum / static_cast<float>(a.N);
+                mu[c] = __double2float_rn(__ddiv_rn(sum, static_cast<double>(a.N)));
                 vmax[c] = mx;
                 vinv[c] = mx > 0.f ? 448.f / mx : 0.f;
             }
@@ -474,7 +486,7 @@ cudaError_t launch_stats_d(const Shape &s, const Src *k, const Src *v, const Sta
     a.vmax_part = ws.vmax_part;
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
     constexpr int RPI = kThreads / (D / 8);
-    const int smem = kStatsStages * 2 * kRowsPerLoad * D * 2 + 2 * RPI * D * 4;
+    const int smem = kStatsStages * 2 * kRowsPerLoad * D * 2 + (kThreads / 32) * D * 8 + RPI * D * 4;
     static std::atomic<uint64_t> limit_set{0};  // one per instantiation
     if ((e = ensure_smem_limit(k_stats<D>, smem, limit_set)) != cudaSuccess) return e;
     const int items = a.nch * s.BH();

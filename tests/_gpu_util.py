@@ -60,15 +60,31 @@ def bf16_step(x: np.ndarray) -> np.ndarray:
     return np.ldexp(1.0, np.floor(np.log2(ax)).astype(np.int64) - 7)
 
 
-def within_tol(got: np.ndarray, want: np.ndarray, rel_tol=REL_L2_TOL, abs_tol=MAX_ABS_TOL):
-    """The parity bar: relative L2 <= rel_tol and every |diff| <= abs_tol, except
-    that where one bf16 step of the reference exceeds abs_tol (|out| >= 2) the
-    two bf16 results may differ by that one step (a rounding decision that
-    fp32-vs-fp64 arithmetic can move).  Returns (ok, rel, max_abs)."""
+# Reading C11: the bar "max |diff| <= 1e-2" is read on the bf16 grid.  Where
+# the oracle's output has |out| >= 2, neighbouring bf16 values are 2^-6 >=
+# 1.56e-2 apart, so an output one rounding decision away from the oracle's
+# (fp32 accumulation on the GPU against fp64 in the oracle moves the value
+# across a rounding midpoint) cannot meet 1e-2 in bf16 whatever the kernel
+# does.  There a difference of exactly one bf16 step is accepted, and at most
+# STEP_FRAC_TOL of the compared elements may use that allowance.
+STEP_FRAC_TOL = 1e-2
+STEP_LOG = []  # (label, elements that used the allowance, elements compared)
+
+
+def within_tol(got: np.ndarray, want: np.ndarray, rel_tol=REL_L2_TOL, abs_tol=MAX_ABS_TOL,
+               step_frac=STEP_FRAC_TOL, label=""):
+    """The parity bar: relative L2 <= rel_tol and every |diff| <= abs_tol,
+    except differences of one bf16 step where that step exceeds abs_tol
+    (reading C11), on at most step_frac of the elements.
+    Returns (ok, rel, max_abs, n_step)."""
     rel, mx = compare(got, want)
-    allow = np.maximum(abs_tol, bf16_step(want) * 1.0001)
-    ok = rel <= rel_tol and bool(np.all(np.abs(got - want) <= allow))
-    return ok, rel, mx
+    diff = np.abs(got - want)
+    over = diff > abs_tol
+    n_step = int(np.count_nonzero(over))
+    one_step = bool(np.all(diff[over] <= bf16_step(want[over]) * 1.0001))
+    ok = rel <= rel_tol and one_step and n_step <= step_frac * max(got.size, 1)
+    STEP_LOG.append((label, n_step, int(got.size)))
+    return ok, rel, mx, n_step
 
 
 def gather(out_gpu: torch.Tensor, heads, rows):

@@ -66,9 +66,9 @@ def test_forward_matches_the_k_residual_oracle(w):
     got = U.bf16_to_f64(out)
     _, bits = oracle.attn_quant(q, k, v, w.sm_scale, k_residual=True)
     want = oracle.bf16_bits_to_f64(bits)
-    ok, rel, mx = U.within_tol(got, want)
+    ok, rel, mx, nstep = U.within_tol(got, want, label="K-residual " + w.name)
     assert np.isfinite(got).all()
-    assert ok, (w.name, rel, mx)
+    assert ok, (w.name, rel, mx, nstep)
 
 
 def test_flux_sampled_rows_and_error_against_exact():
@@ -87,8 +87,8 @@ def test_flux_sampled_rows_and_error_against_exact():
         sl = (slice(b, b + 1), slice(h, h + 1))
         _, bits = oracle.attn_quant(q[sl], k[sl], v[sl], w.sm_scale, rows=rows, k_residual=True)
         want.append(oracle.bf16_bits_to_f64(bits[0, 0]))
-    ok, rel, mx = U.within_tol(got, np.stack(want))
-    assert ok, (rel, mx)
+    ok, rel, mx, nstep = U.within_tol(got, np.stack(want), label="K-residual flux")
+    assert ok, (rel, mx, nstep)
     exact = U.stack(U.oracle_exact_rows(q, k, v, w.sm_scale, heads, rows), heads)
     err_k = U.compare(got, exact)[0]
     err_s = U.compare(U.stack(U.gather(out_s, heads, rows), heads), exact)[0]

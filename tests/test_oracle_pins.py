@@ -13,7 +13,7 @@ import torch
 
 import oracle
 from tests import _brute
-from quantized_attention_qk_b200.inputs import make_qkv, tiny_custom
+from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv, tiny_custom
 
 pytestmark = pytest.mark.usefixtures("oracle_lib")
 
@@ -184,6 +184,30 @@ def test_k_smoothing_statistic_and_blocks():
     ks = k[0, 0].float().numpy() - r["k_mean"][0, 0][None, :]
     deq = kc * np.repeat(r["k_scale"][0, 0], 64)[:200, None]
     assert np.all(np.abs(deq - ks) <= np.repeat(r["k_scale"][0, 0], 64)[:200, None] * 0.5 * (1 + 1e-5))
+
+
+@pytest.mark.parametrize("name,heads", [("tiny", [0, 1]), ("flux", [0, 11, 23]), ("sdxl", [0, 17, 39])])
+def test_k_mean_is_the_exact_mean_on_the_workloads(name, heads):
+    """Reading C1: the K mean is fp32(fp64(exact column sum) / N).  On the
+    workloads every column sum is exact in fp64 whatever the order (a column's
+    values span fewer than 53 bits): the sequential, reversed and 256-token
+    chunked fp64 sums all equal math.fsum, which is why a GPU summing in its
+    own order gets the oracle's mean bit for bit."""
+    w = WORKLOADS[name]
+    q, k, v, _ = make_qkv(w)
+    N = w.N
+    for bh in heads:
+        b, h = divmod(bh, w.H)
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        mu = oracle.quantize(q[sl], k[sl], v[sl])["k_mean"][0, 0]
+        kk = k[b, h].double().numpy()
+        seq = np.cumsum(kk, axis=0)[-1]
+        rev = np.cumsum(kk[::-1], axis=0)[-1]
+        chunks = np.cumsum(np.array([kk[i:i + 256].sum(axis=0) for i in range(0, N, 256)]), axis=0)[-1]
+        for c in range(w.d):
+            exact = math.fsum(kk[:, c])
+            assert seq[c] == exact and rev[c] == exact and chunks[c] == exact, (bh, c)
+            assert mu[c] == np.float32(exact / N), (bh, c)
 
 
 def test_quant_codes_match_numpy_restatement():
