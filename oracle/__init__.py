@@ -68,6 +68,7 @@ def lib():
         L.oracle_e4m3_encode_array.argtypes = [P, I64, P]
         L.oracle_e4m3_decode_array.argtypes = [P, I64, P]
         L.oracle_bf16_rne_array.argtypes = [P, I64, P]
+        L.oracle_s3_exp2_array.argtypes = [P, I64, P]
         for f in ("oracle_attn_exact", "oracle_quantize", "oracle_attn_quant", "oracle_int8_gemm_nt",
                   "oracle_quantize_kres", "oracle_attn_quant_masked", "oracle_block_scores", "oracle_block_select"):
             getattr(L, f).restype = I32
@@ -277,6 +278,14 @@ def e4m3_decode(c) -> np.ndarray:
     x = np.zeros(c.shape, dtype=np.float64)
     lib().oracle_e4m3_decode_array(_ptr(c), c.size, _ptr(x))
     return x
+
+
+def s3_exp2(x) -> np.ndarray:
+    """The fp32 exponential of the selection's masses (reading S3) for x <= 0."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32).ravel())
+    y = np.zeros(x.shape, dtype=np.float32)
+    lib().oracle_s3_exp2_array(_ptr(x), x.size, _ptr(y))
+    return y
 
 
 def bf16_rne(x) -> np.ndarray:

@@ -586,24 +586,56 @@ int oracle_block_scores(const int8_t *qc, const float *qs, const int8_t *kc, con
     return 0;
 }
 
-/* Reading S3 -- which key tiles a query tile keeps.  The estimated softmax
- * mass of key tile j for query tile i is w_ij = n_j * 2^(sbar_ij - max_j
- * sbar_ij) (fp64 here).  The key tiles are ranked by sbar descending, ties by
- * the lower index; the tile at rank t is kept iff the mass of the tiles ranked
- * before it is below tau times the total mass.  So the kept set is the
- * shortest prefix of the ranking whose mass reaches tau of the total; it is
- * never empty, and tau >= 1 keeps every tile.  keep is [nt][nt] (1 = kept). */
+/* Reading S3 -- which key tiles a query tile keeps.  Everything is IEEE fp32
+ * with one rounding per operation, in this order, so that any implementation
+ * following it gets the same bits:
+ *   rank     key tiles by sbar descending, ties by the lower index;
+ *   top      = sbar at rank 0;
+ *   w_t      = float(n_j) * e2(sbar_j - top)  for the tile j at rank t;
+ *   total    = (((0 + w_0) + w_1) + ...)      in rank order;
+ *   lim      = tau * total                    (tau rounded to fp32);
+ *   rank t is kept iff before_t < lim, with before_0 = 0 and
+ *   before_{t+1} = before_t + w_t.
+ * So the kept set is the shortest prefix of the ranking whose mass reaches
+ * tau of the total; rank 0 is always kept, and tau >= 1 keeps every tile.
+ * e2(x) for x <= 0 is 2^x evaluated as: 0 if x < -64 (such a tile weighs
+ * less than 2^-64 of the top one); else k = floor(x), f = x - k, p = the
+ * Taylor polynomial of 2^f = e^(f ln 2) to degree 8 by Horner (coefficients
+ * (ln 2)^i / i! rounded to fp32; p = p*f then p = p + c_i, separately
+ * rounded), and e2 = p * 2^k (exact).  On [0, 1] the polynomial is within
+ * 2e-7 of 2^f; the selection only needs the order of magnitude of each mass,
+ * the fixed arithmetic is what makes it reproducible.  keep is [nt][nt]. */
+static float s3_exp2(float x)
+{
+    if (!(x >= -64.0f)) return 0.0f;
+    float c[9];
+    double fact = 1.0;
+    for (int i = 0; i <= 8; ++i) {
+        if (i > 0) fact *= (double)i;
+        c[i] = (float)(pow(0.69314718055994530942, (double)i) / fact);
+    }
+    const float k = floorf(x);
+    const float f = x - k;
+    float p = c[8];
+    for (int i = 7; i >= 0; --i) {
+        p = p * f;
+        p = p + c[i];
+    }
+    return ldexpf(p, (int)k);
+}
+
 int oracle_block_select(const float *sbar, int N, double tau, uint8_t *keep)
 {
     if (N <= 0 || !(tau > 0.0)) return -1;
+    const float tau32 = (float)tau;
     const int nt = (N + ORACLE_SEL_TILE - 1) / ORACLE_SEL_TILE;
     int *order = (int *)malloc(sizeof(int) * (size_t)nt);
-    double *w = (double *)malloc(sizeof(double) * (size_t)nt);
+    float *w = (float *)malloc(sizeof(float) * (size_t)nt);
     if (!order || !w) { free(order); free(w); return -2; }
     for (int i = 0; i < nt; ++i) {
         const float *row = sbar + (size_t)i * nt;
         uint8_t *kr = keep + (size_t)i * nt;
-        if (tau >= 1.0) {
+        if (tau32 >= 1.0f) {
             for (int j = 0; j < nt; ++j) kr[j] = 1;
             continue;
         }
@@ -616,24 +648,31 @@ int oracle_block_select(const float *sbar, int N, double tau, uint8_t *keep)
             }
             order[t] = j;
         }
-        const double top = (double)row[order[0]];
-        double total = 0.0;
+        const float top = row[order[0]];
+        float total = 0.0f;
         for (int t = 0; t < nt; ++t) {
             const int j = order[t];
             const int nj = (N - j * ORACLE_SEL_TILE) < ORACLE_SEL_TILE ? N - j * ORACLE_SEL_TILE : ORACLE_SEL_TILE;
-            w[t] = (double)nj * exp2((double)row[j] - top);
-            total += w[t];
+            w[t] = (float)nj * s3_exp2(row[j] - top);
+            total = total + w[t];
         }
+        const float lim = tau32 * total;
         for (int j = 0; j < nt; ++j) kr[j] = 0;
-        double before = 0.0;
-        for (int t = 0; t < nt && before < tau * total; ++t) {
+        float before = 0.0f;
+        for (int t = 0; t < nt && before < lim; ++t) {
             kr[order[t]] = 1;
-            before += w[t];
+            before = before + w[t];
         }
     }
     free(order);
     free(w);
     return 0;
+}
+
+/* Array form of the selection's exponential, for the tests. */
+void oracle_s3_exp2_array(const float *x, int64_t n, float *y)
+{
+    for (int64_t i = 0; i < n; ++i) y[i] = s3_exp2(x[i]);
 }
 
 /* Integer score tile from given codes: s[i][j] = sum_c a[i][c] * b[j][c]

@@ -9,7 +9,10 @@
 //       evaluated in fp32 in a fixed order from exact integer code sums;
 //   S3  query tile i keeps the shortest prefix of its key tiles ranked by
 //       score (ties: lower index first) whose estimated mass
-//       n_j 2^(score - max score) reaches tau of the total (tau >= 1: all);
+//       n_j 2^(score - max score) reaches tau of the total (tau >= 1: all),
+//       in fp32 with one rounding per operation in a fixed order (masses by
+//       a fixed Taylor polynomial, sums in rank order), so that the kept set
+//       is reproducible bit for bit;
 //   S4  tau(step) moves linearly from tau_start to tau_end over the steps.
 #include <cuda_runtime.h>
 
@@ -119,18 +122,35 @@ __global__ void __launch_bounds__(kScoreThreads)
     sbar[((size_t)bh * nt + i) * nt + j] = __fdiv_rn(__fmul_rn(acc, s_l2), static_cast<float>(ni * nj));
 }
 
+// 2^x for x <= 0 as reading S3 fixes it: 0 below -64; else k = floor(x),
+// f = x - k, the degree-8 Taylor polynomial of 2^f = e^(f ln 2) by Horner with
+// the coefficients (ln 2)^i / i! rounded to fp32 (each multiply and add rounded
+// on its own), times 2^k (exact: the result stays a normal number).
+__device__ __forceinline__ float s3_exp2(float x) {
+    if (!(x >= -64.f)) return 0.f;
+    const float c[9] = {0x1p+0f,          0x1.62e43p-1f,    0x1.ebfbep-3f,  0x1.c6b08ep-5f, 0x1.3b2ab6p-7f,
+                        0x1.5d87fep-10f,  0x1.430912p-13f,  0x1.ffcbfcp-17f, 0x1.62c022p-20f};
+    const float k = floorf(x);
+    const float f = __fsub_rn(x, k);
+    float p = c[8];
+#pragma unroll
+    for (int i = 7; i >= 0; --i) p = __fadd_rn(__fmul_rn(p, f), c[i]);
+    return __fmul_rn(p, __int_as_float((127 + static_cast<int>(k)) << 23));
+}
+
 // One CTA per (b,h, query tile i): ranks the row's key tiles (bitonic sort of
 // P >= nt entries in shared memory: higher score first, then lower index),
-// computes their masses n_j 2^(score - top) in parallel, and keeps the ranks
-// whose preceding mass is below tau of the total (reading S3): a fixed-order
-// block scan (each thread sums its own contiguous ranks, then the thread
-// totals are scanned) gives the preceding masses.  Writes the row's mask words.
+// computes their masses n_j 2^(score - top) in parallel, then one thread takes
+// the total and the kept prefix in rank order (reading S3's fixed fp32
+// order: rank t is kept while the mass ranked before it is below tau of the
+// total).  Writes the row's mask words.
 __global__ void __launch_bounds__(kSelThreads)
     k_select(const float *__restrict__ sbar, int N, int nt, int P, int words, float tau, uint32_t *__restrict__ mask) {
     extern __shared__ float sm[];
     float *key = sm;                                       // [P] score, then mass
     int *idx = reinterpret_cast<int *>(key + P);           // [P] key tile
     uint32_t *mw = reinterpret_cast<uint32_t *>(idx + P);  // [words]
+    __shared__ int s_cut;
     const int i = blockIdx.x, bh = blockIdx.y;
     const float *row = sbar + ((size_t)bh * nt + i) * nt;
     for (int w = threadIdx.x; w < words; w += kSelThreads) mw[w] = 0u;
@@ -161,47 +181,23 @@ __global__ void __launch_bounds__(kSelThreads)
         }
         const float top = key[0];
         __syncthreads();
-        // masses, and each thread's sum over its contiguous ranks
-        const int per = (nt + kSelThreads - 1) / kSelThreads;
-        const int r0 = threadIdx.x * per, r1 = min(nt, r0 + per);
-        float own = 0.f;
-        for (int r = r0; r < r1; ++r) {
+        for (int r = threadIdx.x; r < nt; r += kSelThreads) {
             const int j = idx[r];
-            const float w = static_cast<float>(min(kKvTile, N - j * kKvTile)) * exp2f(key[r] - top);
-            key[r] = w;
-            own += w;
+            key[r] = __fmul_rn(static_cast<float>(min(kKvTile, N - j * kKvTile)), s3_exp2(__fsub_rn(key[r], top)));
         }
-        // exclusive scan of the thread sums in thread order: within each warp by
-        // shuffles, then over the warp totals
-        const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-        float incl = own;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const float o = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d) incl += o;
-        }
-        __shared__ float wsum[kSelThreads / 32];
-        __shared__ float s_total;
-        if (lane == 31) wsum[wid] = incl;
         __syncthreads();
         if (threadIdx.x == 0) {
-            float run = 0.f;
-            for (int w = 0; w < kSelThreads / 32; ++w) {
-                const float v = wsum[w];
-                wsum[w] = run;
-                run += v;
-            }
-            s_total = run;
+            float total = 0.f;
+#pragma unroll 8
+            for (int r = 0; r < nt; ++r) total = __fadd_rn(total, key[r]);
+            const float lim = __fmul_rn(tau, total);
+            float before = 0.f;
+            int cut = 0;
+            while (cut < nt && before < lim) before = __fadd_rn(before, key[cut++]);
+            s_cut = cut;
         }
         __syncthreads();
-        // rank r is kept iff the mass ranked before it is below tau of the total
-        const float lim = tau * s_total;
-        float before = wsum[wid] + (incl - own);
-        for (int r = r0; r < r1 && before < lim; ++r) {
-            const int j = idx[r];
-            atomicOr(&mw[j >> 5], 1u << (j & 31));
-            before += key[r];
-        }
+        for (int r = threadIdx.x; r < s_cut; r += kSelThreads) atomicOr(&mw[idx[r] >> 5], 1u << (idx[r] & 31));
     }
     __syncthreads();
     for (int w = threadIdx.x; w < words; w += kSelThreads) mask[((size_t)bh * nt + i) * words + w] = mw[w];
