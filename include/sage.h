@@ -49,6 +49,9 @@
  *     with respect to other work on `stream` is the ordinary stream order.
  *   - N_pad = ceil(N/128)*128.  Padded rows of every code buffer are written
  *     as zeros; padded blocks get scale 0.
+ *   - Device tensors must live on the current device (checked on the first
+ *     input and the output: SAGE_ERR_INVALID_ARG otherwise); kernels launch on
+ *     the current device.
  *   - Every device buffer is owned by the caller; the library keeps no pointer
  *     after a call returns.  Calls are asynchronous on `stream` and return
  *     after the launches.  A kernel that gives up waiting on an internal
@@ -95,13 +98,18 @@ sage_status_t sage_check(sage_stream_t stream);
 size_t sage_attn_workspace_bytes(int B, int H, int N, int d);
 
 /* Bytes of scratch sage_quant_qk / sage_quant_v need (the per-chunk partial
- * statistics of the smoothing mean and of the V channel maxima). */
+ * statistics of the smoothing mean and of the V channel maxima): with
+ * C = ceil(N/256) chunks and up(x) = x rounded up to 1024,
+ *   up(8*B*H*C*d) + up(4*B*H*C*d) + 2*up(4*B*H*d)
+ * (fp64 K sums and fp32 V maxima per chunk, then the fp32 K mean and V factor
+ * per head); 0 for an invalid shape. */
 size_t sage_quant_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * sage_quant_qk -- smoothing plus block quantization of Q and K ([H3] section 一;
  * readings C1-C3).
- *   k_mean[b,h,c] = (1/N) sum_n K[b,h,n,c]                 (fp32 accumulation)
+ *   k_mean[b,h,c] = fp32( (sum_n K[b,h,n,c]) / N )   (the sum in fp64, exact
+ *       whenever a column's values span fewer than 53 bits; one fp64 division)
  *   Q, per 128-token block:  amax = max|Q| over the block's valid tokens and all
  *       channels; q_scale = amax/127; q_i8 = rne(Q * (127/amax)) in [-127,127]
  *   K, the same per 64-token block on (K - k_mean).
@@ -131,10 +139,15 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4],
  *   workspace.  The statistics scratch is a fixed array of
  *   SAGE_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library's device memory;
  *   every GPU that loads the library holds it until the process exits.  A shape
- *   whose scratch (sage_quant_workspace_bytes) exceeds it is rejected with
- *   SAGE_ERR_WORKSPACE before anything is launched.  The call allocates nothing.
+ *   whose scratch (sage_quant_workspace_bytes, about 12*B*H*d*ceil(N/256)
+ *   bytes) exceeds it is rejected with SAGE_ERR_WORKSPACE before anything is
+ *   launched: e.g. (1,24,4608,128) needs 0.69 MB and (1,24,16384,128) 2.4 MB
+ *   and fit, (1,40,34020,128) needs 8.2 MB and (1,24,65536,128) 9.5 MB and do
+ *   not.  The inputs must be on the current device (SAGE_ERR_INVALID_ARG
+ *   otherwise).  The call allocates nothing.
  *   The first call on each device looks up the array's device address (with
- *   that device current); make that first call before any stream capture.
+ *   that device current) and keeps it; make that first call before any stream
+ *   capture, and do not go on using the library after cudaDeviceReset.
  *   All calls on a device share the array: calls that may overlap on the GPU
  *   (different streams without ordering) race and must be serialized by the
  *   caller.  The array keeps the last call's contents; nothing in it needs to

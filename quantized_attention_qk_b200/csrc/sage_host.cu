@@ -129,12 +129,37 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
         owned = true;
     }
     Events ev;
+    bool forked = false;  // the internal streams wait on the caller's stream
+    // Every return from here on goes through finish(): once the internal
+    // streams took work, the caller's stream is made to wait for all of them
+    // (also after an error, so that no copy into out_host or read of scratch
+    // is still pending when the caller's stream moves on), and an owned
+    // scratch is freed in stream order.  The first error is the one reported.
+    auto finish = [&](sage_status_t status, cudaError_t err, const char *what) -> sage_status_t {
+        if (status != SAGE_OK) cuda_fail(err, what);
+        if (forked) {
+            for (int i = 0; i < kStreams; ++i) {
+                cudaError_t x = cudaEventRecord(ev.ev[1 + i], st[i]);
+                if (x == cudaSuccess) x = cudaStreamWaitEvent(user, ev.ev[1 + i], 0);
+                if (x != cudaSuccess && status == SAGE_OK) status = cuda_fail(x, "joining the internal streams");
+            }
+        }
+        if (owned) {
+            cudaError_t x = cudaFreeAsync(scratch, user);
+            if (x != cudaSuccess && status == SAGE_OK) status = cuda_fail(x, "cudaFreeAsync(scratch)");
+        }
+        return status;
+    };
     for (cudaEvent_t &x : ev.ev)
-        if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e, "event");
+        if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess)
+            return finish(SAGE_ERR_CUDA, e, "event");
     // the internal streams start after everything already on the caller's stream
-    if ((e = cudaEventRecord(ev.ev[0], user)) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    for (int i = 0; i < kStreams; ++i)
-        if ((e = cudaStreamWaitEvent(st[i], ev.ev[0], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    if ((e = cudaEventRecord(ev.ev[0], user)) != cudaSuccess) return finish(SAGE_ERR_CUDA, e, "cudaEventRecord");
+    for (int i = 0; i < kStreams; ++i) {
+        if ((e = cudaStreamWaitEvent(st[i], ev.ev[0], 0)) != cudaSuccess)
+            return finish(SAGE_ERR_CUDA, e, "cudaStreamWaitEvent");
+        forked = true;
+    }
 
     const size_t elems = (size_t)B * H * N * d;
     char *base = static_cast<char *>(scratch);
@@ -162,7 +187,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
                     const int64_t off = boff + x * hd + (int64_t)h0 * d;
                     e = cudaMemcpy2DAsync(d_in + off, row * 2, h_in + off, row * 2, (size_t)hc * d * 2, N,
                                           cudaMemcpyHostToDevice, s);
-                    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+                    if (e != cudaSuccess) return finish(SAGE_ERR_CUDA, e, "host-to-device copy");
                 }
                 const uint16_t *p0 = d_in + boff + (int64_t)h0 * d;
                 q = Src{p0, (int64_t)N * row, d, row};
@@ -174,7 +199,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
                 for (int x = 0; x < 3; ++x) {
                     e = cudaMemcpyAsync(d_in + x * elems + off, h_in + x * elems + off, (size_t)hc * nd * 2,
                                         cudaMemcpyHostToDevice, s);
-                    if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+                    if (e != cudaSuccess) return finish(SAGE_ERR_CUDA, e, "host-to-device copy");
                 }
                 q = Src{d_in + off, (int64_t)H * nd, nd, d};
                 k = Src{d_in + elems + off, (int64_t)H * nd, nd, d};
@@ -184,21 +209,18 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
             const Dst o{d_out + ooff, (int64_t)H * nd, nd, d};
             const Codes codes = carve_codes(ws, cs);
             const StatsWs sw = carve_stats_ws(ws + up(codes_bytes(cs)), cs);
-            if ((e = launch_stats(cs, &k, &v, sw, s)) != cudaSuccess) return cuda_fail(e, "statistics pass");
+            if ((e = launch_stats(cs, &k, &v, sw, s)) != cudaSuccess)
+                return finish(SAGE_ERR_CUDA, e, "statistics pass");
             if ((e = launch_quant(cs, &q, &k, &v, sw, nullptr, codes, s)) != cudaSuccess)
-                return cuda_fail(e, "quantize pass");
-            if ((e = launch_attention(cs, codes, o, sm_scale, s)) != cudaSuccess) return cuda_fail(e, "attention kernel");
+                return finish(SAGE_ERR_CUDA, e, "quantize pass");
+            if ((e = launch_attention(cs, codes, o, sm_scale, s)) != cudaSuccess)
+                return finish(SAGE_ERR_CUDA, e, "attention kernel");
             if ((e = cudaMemcpyAsync(h_out + ooff, d_out + ooff, (size_t)hc * nd * 2, cudaMemcpyDeviceToHost, s)) !=
                 cudaSuccess)
-                return cuda_fail(e, "device-to-host copy");
+                return finish(SAGE_ERR_CUDA, e, "device-to-host copy");
         }
-    // the caller's stream continues after both internal streams
-    for (int i = 0; i < kStreams; ++i) {
-        if ((e = cudaEventRecord(ev.ev[1 + i], st[i])) != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-        if ((e = cudaStreamWaitEvent(user, ev.ev[1 + i], 0)) != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
-    }
-    if (owned && (e = cudaFreeAsync(scratch, user)) != cudaSuccess) return cuda_fail(e, "cudaFreeAsync(scratch)");
-    return SAGE_OK;
+    // the caller's stream continues after all internal streams
+    return finish(SAGE_OK, cudaSuccess, nullptr);
 }
 
 }  // extern "C"

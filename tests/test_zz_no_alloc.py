@@ -34,6 +34,26 @@ def test_noalloc_rejects_a_shape_beyond_its_scratch(L):
     assert b"scratch" in L.sage_last_error_message()
 
 
+def test_noalloc_scratch_bound_on_the_workloads(L):
+    """The scratch a shape needs is the documented formula; the video and 64K
+    workloads need more than the 4 MiB array and are rejected with status 3
+    (before any launch), the smaller ones fit."""
+    up = lambda x: -(-x // 1024) * 1024
+    for name, w in WORKLOADS.items():
+        C = -(-w.N // 256)
+        need = up(8 * w.B * w.H * C * w.d) + up(4 * w.B * w.H * C * w.d) + 2 * up(4 * w.B * w.H * w.d)
+        assert sage.sage_quant_workspace_bytes(w.B, w.H, w.N, w.d) == need, name
+        assert (need <= 4 << 20) == (name not in ("video", "long64k")), name
+    w = WORKLOADS["video"]
+    st = (ctypes.c_int64 * 4)(w.N * 3 * w.H * w.d, w.d, 3 * w.H * w.d, 1)
+    p = ctypes.c_void_p(16 * 4096)
+    rc = L.sage_quant_qk_noalloc(p, st, p, st, w.B, w.H, w.N, w.d, p, p, p, p, None, None)
+    assert rc == 3
+    assert b"scratch" in L.sage_last_error_message()
+    # a shape the library does not take at all is reported as such, not as scratch
+    assert L.sage_quant_qk_noalloc(p, st, p, st, 1, 70000, 128, 128, p, p, p, p, None, None) == 2
+
+
 @pytest.mark.gpu
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs a CUDA device")
 def test_noalloc_matches_the_workspace_entry_point_twice(L):
