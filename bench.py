@@ -5,11 +5,17 @@ One step = one full forward (statistics + quantize + fused attention) of the
 workload, through the C ABI (sage_attn_fwd).  Metric: TOPS = 4*B*H*N^2*d / t.
 
   python bench.py [--gpus N --steps K --warmup W] [--workload flux|video|...]
+  python bench.py --shard ...            # one problem split by heads over the GPUs
   python bench.py --impl reference ...   # the CPU oracle, timed on the host
 
 N > 1 GPUs (torchrun): every rank runs its own copy of the workload (the heads
 of independent problems; no data-path collective), so the scaling is weak and
 the value is the sum over ranks of the work divided by the slowest rank's time.
+
+With --shard the ranks instead split ONE problem by heads (each rank computes
+its heads on strided views of the shared input) and all-gather the bf16
+outputs over NCCL, so the scaling is strong; the time of a step covers the
+kernels and the gather.
 
 Inputs are seeded synthetic tensors (quantized_attention_qk_b200.inputs).  The
 L2 is flushed (a 256 MB write) before every timed step, outside the events.
@@ -395,6 +401,62 @@ def run_gpu(args):
     reps.close()
 
 
+# --------------------------------------------------------------------------- head-sharded arm
+def run_shard(args):
+    """One problem split by heads over the ranks (replicas.sharded_forward with
+    the NCCL all-gather), timed on the device, the maximum over ranks."""
+    import torch
+
+    import quantized_attention_qk_b200 as sage
+    from quantized_attention_qk_b200 import build as sage_build
+    from quantized_attention_qk_b200.inputs import WORKLOADS, make_qkv
+    from quantized_attention_qk_b200.replicas import Replicas, env_int, head_range, timed_sharded
+
+    world = env_int("WORLD_SIZE", 1)
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    if not torch.cuda.is_available():
+        raise SystemExit("no CUDA device")
+    local = env_int("LOCAL_RANK", 0)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    reps = Replicas(device=dev)
+    sage_build.build()
+    sage.lib()
+    w = WORKLOADS[args.workload]
+    q, k, v, bufs = make_qkv(w, device=dev)          # every rank holds the whole input
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    clk = ClockSampler(dev)
+    clk.start()
+    out, mine, total = timed_sharded(q, k, v, reps, args.steps, args.warmup, sm_scale=w.sm_scale,
+                                     before_step=flush.zero_)
+    clocks = clk.stop()
+    sage.sage_check()
+    # outside the timed region: the gathered result against the whole forward on this rank
+    whole = sage.sage_attn_fwd(q, k, v, sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    same = bool(torch.equal(out.view(torch.int16), whole.view(torch.int16)))
+    same_all = reps.max(0.0 if same else 1.0) == 0.0
+    h0, h1 = head_range(w.H, world, reps.rank)
+    value = w.ops * args.steps / (total * 1e-3) / 1e12
+    line = {"metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(total / args.steps, 4), "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": DTYPE,
+            "data": "synthetic (seeded N(0,1) Q/K/V, K bias and outlier channels)",
+            "config": {"workload": _workload_desc(w), "B": w.B, "H": w.H, "N": w.N, "d": w.d, "layout": w.layout,
+                       "parallelism": f"heads split over {world} GPU(s) (rank 0: heads {h0}..{h1 - 1}), "
+                                      "bf16 outputs all-gathered over NCCL" + (" (no gather at one GPU)" if world == 1
+                                                                              else ""),
+                       "l2": "flushed before every timed step (256 MB write, outside the events)",
+                       "timing": "CUDA events on each rank's stream around forward + gather; max over ranks"},
+            "gathered_equals_whole_forward": same_all,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clocks}
+    if reps.rank == 0:
+        print(json.dumps(line, ensure_ascii=False), flush=True)
+    del q, k, v, bufs, out, whole
+    reps.close()
+
+
 # --------------------------------------------------------------------------- reference arm (the CPU oracle)
 def run_reference(args):
     from quantized_attention_qk_b200.inputs import WORKLOADS
@@ -442,11 +504,15 @@ def main():
                     help="time the K-residual forward instead of the smoothing one")
     ap.add_argument("--fused-q", dest="fused_q", action="store_true",
                     help="time the forward that quantizes Q in the attention kernel's prologue")
+    ap.add_argument("--shard", action="store_true",
+                    help="split one problem by heads over the GPUs and all-gather the outputs (strong scaling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.shard:
+        run_shard(args)
     else:
         run_gpu(args)
 

@@ -124,3 +124,44 @@ def sharded_forward(q, k, v, reps: Replicas, sm_scale=None, gather: bool = True,
         a, b = head_range(H, reps.world, r)
         out[:, a:b] = parts[r][:, : b - a]
     return out
+
+
+def timed_sharded(q, k, v, reps: Replicas, steps: int, warmup: int, sm_scale=None, attn=None, out_dtype=None,
+                  before_step=None):
+    """Time `steps` head-sharded forwards of one problem (each with the
+    all-gather) after `warmup` untimed ones.  On CUDA tensors each step is
+    timed with events on the current stream (which waits for the collective);
+    on CPU tensors with the host clock.  `before_step` (e.g. an L2 flush) runs
+    before every timed step, outside its timing.  Every rank takes the same
+    collective steps.  Returns (the last gathered output, this rank's total
+    ms, the maximum of the totals over the ranks)."""
+    import time
+
+    cuda = q.is_cuda
+    out = None
+    for _ in range(warmup):
+        out = sharded_forward(q, k, v, reps, sm_scale=sm_scale, attn=attn, out_dtype=out_dtype)
+    if cuda:
+        torch.cuda.synchronize()
+    reps.barrier()
+    if cuda:
+        torch.cuda.synchronize()
+    total = 0.0
+    for _ in range(steps):
+        if before_step is not None:
+            before_step()
+        if cuda:
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            out = sharded_forward(q, k, v, reps, sm_scale=sm_scale, attn=attn, out_dtype=out_dtype)
+            e1.record()
+            e1.synchronize()
+            total += e0.elapsed_time(e1)
+        else:
+            t0 = time.perf_counter()
+            out = sharded_forward(q, k, v, reps, sm_scale=sm_scale, attn=attn, out_dtype=out_dtype)
+            total += (time.perf_counter() - t0) * 1e3
+    if cuda:
+        torch.cuda.synchronize()
+    reps.barrier()
+    return out, total, reps.max(total)

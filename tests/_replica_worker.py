@@ -6,7 +6,8 @@ import sys
 
 sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
 
-from quantized_attention_qk_b200.replicas import Replicas, env_int, head_range, sharded_forward, whole_job_tops  # noqa: E402
+from quantized_attention_qk_b200.replicas import (Replicas, env_int, head_range, sharded_forward,  # noqa: E402
+                                                  timed_sharded, whole_job_tops)
 
 
 def main():
@@ -43,6 +44,24 @@ def main():
             result["gathered_equal"] = bool(torch.equal(full, ref))
             result["part_equal"] = bool(torch.equal(part, ref[:, h0:h1]))
             result["heads"] = [h0, h1]
+        elif mode == "timed_shard":
+            # the timing path of bench.py --shard on CPU: warm-up, timed steps,
+            # the maximum over ranks, and the gathered output
+            import torch
+            import oracle
+            g = torch.Generator().manual_seed(6)
+            q, k, v = (torch.randn(1, 5, 32, 16, generator=g).to(torch.bfloat16) for _ in range(3))
+
+            def attn(qs, ks, vs, sm_scale=None):
+                return torch.from_numpy(oracle.attn_exact(qs, ks, vs, sm_scale))
+
+            calls = []
+            got, mine, mx = timed_sharded(q, k, v, reps, steps=3, warmup=3, sm_scale=0.25, attn=attn,
+                                          out_dtype=torch.float64, before_step=lambda: calls.append(1))
+            result["gathered_equal"] = bool(torch.equal(got, attn(q, k, v, sm_scale=0.25)))
+            result["mine_ms"] = mine
+            result["max_ms"] = mx
+            result["before_step_calls"] = len(calls)
         elif mode == "die":
             if rank == 1:
                 os._exit(3)  # leaves between steps, before the next collective

@@ -113,3 +113,15 @@ def test_head_sharded_forward_gathers_the_whole_result(tmp_path, world, H):
     for r in res:
         assert "error" not in r, r
         assert r["gathered_equal"] and r["part_equal"], r
+
+
+def test_timed_head_sharding_takes_the_slowest_rank(tmp_path):
+    """bench.py --shard's timing path over two gloo ranks: both ranks time the
+    same steps, report the same maximum, which is at least their own time, and
+    the gathered output is the whole problem's."""
+    codes, res = _run_ranks("timed_shard", tmp_path)
+    assert codes == [0, 0], res
+    assert all(r.get("error") is None for r in res), res
+    assert all(r["gathered_equal"] for r in res)
+    assert res[0]["max_ms"] == res[1]["max_ms"] == max(r["mine_ms"] for r in res)
+    assert all(r["before_step_calls"] == 3 for r in res)
