@@ -359,7 +359,7 @@ def run_gpu(args):
                 "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
                        "attention, bf16 out -> pinned host; dense)"},
         "gpu_launches": (LAUNCHES_PER_STEP + (3 if args.tau is not None and args.tau < 1 else 0) +
-                         (2 if args.kres else 0)) * args.steps,
+                         (1 if args.kres else 0)) * args.steps,
         "clocks": r["clocks"],
     }
     if args.tau is not None:

@@ -364,18 +364,24 @@ sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4
                                     int8_t *k_i8, float *k_scale, uint16_t *k_bmean,
                                     sage_stream_t stream);
 
-/* Bytes of scratch sage_attn_fwd_kres needs (0 for a shape rejected): the
- * codes, the V statistics, the bf16 block means and the fp32 mean term
- * ([B*H][N_pad/64][N_pad], 4*B*H*N_pad^2/64 bytes). */
+/* Bytes of scratch sage_attn_fwd_kres needs on the current device (0 for a
+ * shape rejected, or when the device cannot be queried): the codes, the V
+ * statistics, the bf16 block means and the attention kernel's per-SM scratch
+ * slots for the mean term ([SMs][N_pad/64][256] fp32: 1 KiB per SM and
+ * 64-token block, linear in N). */
 size_t sage_attn_kres_workspace_bytes(int B, int H, int N, int d);
 
 /*
  * sage_attn_fwd_kres -- the forward with K-residual quantization instead of
  * the smoothing: Q and V coded as in sage_attn_fwd, K as in
- * sage_quant_k_residual, the mean term computed on the tensor cores (bf16
- * products, fp32 accumulation), and the fused attention kernel adding it to
- * each score's exponent.  Arguments, layouts, events and errors as
- * sage_attn_fwd_ev.
+ * sage_quant_k_residual, and the fused attention kernel adding the mean term
+ * to each score's exponent.  Each attention CTA computes the mean term of its
+ * 256 query rows against every 64-token block first, on the tensor cores
+ * (tcgen05 kind::f16: bf16 Q rows times bf16 block means, fp32 accumulation,
+ * times fp32(sm_scale * log2 e)), and keeps it in the scratch slot of the SM
+ * it runs on.  Arguments, layouts, events and errors as sage_attn_fwd_ev;
+ * the workspace is sage_attn_kres_workspace_bytes for the device the call
+ * runs on.
  */
 sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4],
                                  const void *k, const int64_t k_stride[4],

@@ -458,12 +458,14 @@ sage_status_t sage_attn_fwd_fused_q(const void *q, const int64_t q_stride[4], co
 }
 
 static size_t kres_bmean_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.d * 2); }
-static size_t kres_ebias_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_kblocks() * s.n_pad() * 4); }
+// per-SM scratch slots of the attention kernel's mean term: [SMs][nkb][256] fp32
+static size_t kres_slot_bytes(const Shape &s) { return up((size_t)kres_slots() * s.n_kblocks() * 256 * 4); }
 
 size_t sage_attn_kres_workspace_bytes(int B, int H, int N, int d) {
     if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
     const Shape s{B, H, N, d};
-    return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + kres_bmean_bytes(s) + kres_ebias_bytes(s);
+    if (kres_slots() <= 0) return 0;
+    return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + kres_bmean_bytes(s) + kres_slot_bytes(s);
 }
 
 sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4], int B, int H, int N, int d,
@@ -492,24 +494,25 @@ sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4], const
         return r;
     const Shape s{B, H, N, d};
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int n_slots = kres_slots();
+    if (n_slots <= 0) return fail(SAGE_ERR_CUDA, "could not read the device's SM count");
     Scratch scr;
     const size_t cb = up(codes_bytes(s)), sb = up(stats_ws_bytes(s)), mb = kres_bmean_bytes(s);
-    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + sb + mb + kres_ebias_bytes(s), st))) return r;
+    if ((r = get_scratch(scr, workspace, workspace_bytes, cb + sb + mb + kres_slot_bytes(s), st))) return r;
     char *base = static_cast<char *>(scr.ptr);
     const Codes c = carve_codes(base, s);
     const StatsWs ws = carve_stats_ws(base + cb, s);
     uint16_t *bmean = reinterpret_cast<uint16_t *>(base + cb + sb);
-    float *ebias = reinterpret_cast<float *>(base + cb + sb + mb);
+    float *eslot = reinterpret_cast<float *>(base + cb + sb + mb);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
     cudaError_t e = launch_stats(s, nullptr, &vs, ws, st);
     if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
     if ((e = launch_quant(s, &qs, nullptr, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
     if ((e = launch_kres(s, ks, c.k_i8, c.k_scale, bmean, st)) != cudaSuccess)
         return cuda_fail(e, "K-residual quantization");
-    if ((e = launch_ebias(s, qs, bmean, sm_scale, ebias, st)) != cudaSuccess) return cuda_fail(e, "mean term");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");
-    if ((e = launch_attention_kres(s, c, dst(out, o_stride), sm_scale, ebias, st)) != cudaSuccess)
+    if ((e = launch_attention_kres(s, c, qs, bmean, dst(out, o_stride), sm_scale, eslot, n_slots, st)) != cudaSuccess)
         return cuda_fail(e, "attention kernel");
     if (attn_end && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_end), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");

@@ -42,10 +42,20 @@
 // the quantize pass codes K and V only.  No P is stored before S(0), which
 // waits for all eight warps' codes.
 // K-residual instantiation (KRES): K holds the codes of its residual inside
-// each 64-token block, and every score gains that block's mean term e[row][b]
-// (precomputed in fp32, block-major so a warp's rows read it coalesced); each
-// 128-key step covers two blocks, so e folds into the two per-half offsets
-// the exponent already takes (no work per score).
+// each 64-token block, and every score gains that block's mean term
+// e[row][b] = (q_row . mean_b) * sm_scale * log2 e; each 128-key step covers
+// two blocks, so e folds into the two per-half offsets the exponent already
+// takes (no work per score).  The CTA computes e for its 256 rows and every
+// block in a prologue, while tensor memory and the ring / P buffers are still
+// free: the producer loads the tiles' bf16 Q rows (into the ring's last two
+// stages) and up to 256 block means at a time (into the P buffers; 128-byte
+// swizzle) while the ring's first stage takes K/V tiles, the MMA warp
+// multiplies them on the tensor cores (tcgen05 kind::f16, bf16 x bf16 ->
+// fp32, M = 128, N <= 256, one accumulator per tile), and the softmax warps
+// scale each row's values and keep them in a
+// per-SM scratch slot [block][256 rows] (one CTA per SM at a time, so the
+// slot of the SM the CTA runs on is its own), which the same threads read back
+// one step ahead in the main loop.
 // Numerics (readings C4-C8): x = S*(sq*sm_scale*log2e*sk) with one sk per
 // 64-key block; running max m' = max(m, ceil(rowmax x)) so that the O / l
 // rescale 2^(m-m') is an exact power of two; P = e4m3(2^(x-m') * 448) computed as
@@ -84,7 +94,7 @@ struct Cfg {
     static constexpr int THREADS = 384;            // three warpgroups
     static constexpr int LAUNCH_REGS = 168;        // per thread, what 384 threads x 1 block allow
     static constexpr uint32_t SOFTMAX_REGS = 216;  // warpgroups 0 and 1 after setmaxnreg
-    static constexpr uint32_t OTHER_REGS = 64;     // warpgroup 2 (TMA, MMA, two idle warps)
+    static constexpr uint32_t OTHER_REGS = 72;     // warpgroup 2 (TMA, MMA, two idle warps)
     static_assert(2 * 128 * SOFTMAX_REGS + 128 * OTHER_REGS <= LAUNCH_REGS * THREADS,
                   "register split exceeds the registers the block is launched with");
 };
@@ -102,6 +112,9 @@ struct Ctl {
     uint64_t drain;
     uint64_t qb_full;       // FUSED_Q: the bf16 Q rows landed
     uint64_t q_amax_bar[2]; // FUSED_Q, per tile: the four warps posted their |max|
+    uint64_t mb_full[1];    // KRES prologue: a chunk of block means landed
+    uint64_t e_full[1];     // KRES prologue: a chunk's mean-term products are in tensor memory
+    uint64_t e_free[1];     // KRES prologue: the softmax warps took them out
     float q_amax[2][4];
     int steps[3];           // SPARSE: own steps of tile 0, of tile 1, union steps
     uint32_t tmem_base;
@@ -133,9 +146,10 @@ struct AttnParams {
     // query tile i attends to key tile j
     const uint32_t *kv_mask;
     int mask_words;
-    // KRES instantiation: mean term of every (K block, query row), [BH][nkb][N_pad]
-    const float *ebias;
-    int q_swap;            // FUSED_Q: the bf16 Q map takes H before N
+    // KRES instantiation: per-SM scratch slots of the mean term, [n_slots][nkb][256]
+    float *eslot;
+    int n_slots;
+    int q_swap;            // FUSED_Q, KRES: the bf16 Q map takes H before N
 };
 
 // Step lists of the SPARSE instantiation, built by one warp from mask rows r0
@@ -281,7 +295,8 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 template <int D, bool EXPORT_S, bool SPARSE, bool KRES, bool FUSED_Q>
 __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
     k_attn(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qb, const AttnParams p) {
+           const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qb,
+           const __grid_constant__ CUtensorMap tm_mean, const AttnParams p) {
     using C = Cfg<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -319,6 +334,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
             mbar_init(&ctl->o_final[t], 1);
         }
         mbar_init(&ctl->drain, 1);
+        mbar_init(&ctl->mb_full[0], 1);
+        mbar_init(&ctl->e_full[0], 1);
+        mbar_init(&ctl->e_free[0], 8);
         ctl->abort.flag = 0;
         fence_barrier_init();
     }
@@ -326,7 +344,22 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         tma_prefetch_desc(FUSED_Q ? &tm_qb : &tm_q);
         tma_prefetch_desc(&tm_k);
         if (!EXPORT_S) tma_prefetch_desc(&tm_v);
+        if (KRES) {
+            tma_prefetch_desc(&tm_qb);
+            tma_prefetch_desc(&tm_mean);
+        }
     }
+    // KRES prologue: chunks of up to 256 K blocks (one MMA per tile and K step,
+    // tile t's products at tensor-memory columns [256 t, 256 t + 256)); the
+    // chunk's means sit in the P buffers ([channel half][256 blocks][64]), the
+    // bf16 Q rows of tile t in the ring's stages 1 and 2 (its K slots for tile
+    // 0, its V slots for tile 1: [channel half][128 rows][64]), so stage 0
+    // takes the first K/V tiles meanwhile
+    constexpr int kEChunk = 256;
+    uint8_t *const sQb[2] = {sK + C::K_BYTES, sV + C::V_BYTES};
+    static_assert(2 * C::K_BYTES == C::BM * D * 2 && kEChunk * D * 2 <= 4 * C::P_BYTES,
+                  "the prologue's operands fit the ring's last stages and the P buffers");
+    const int e_chunks = KRES ? (p.nkb + kEChunk - 1) / kEChunk : 0;
     // everything below reads what the previous kernel of the stream wrote
     grid_dep_wait();
     for (int i = threadIdx.x; i < D; i += blockDim.x) ctl->v_scale[i] = EXPORT_S ? 0.f : p.v_scale[bh * D + i];
@@ -373,22 +406,64 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 tma_load_3d(sQ, &tm_q, &ctl->q_full, 0, qt0 * C::BM, bh);
                 tma_load_3d(sQ + C::Q_BYTES, &tm_q, &ctl->q_full, 0, (qt0 + 1) * C::BM, bh);
             }
+            bool pro_ok = true;
+            int m_issued = 0;  // KRES: means chunks issued
             int issued = 0;
-            const int nsteps = SPARSE ? ctl->steps[2] : nkv;
-            for (int j = 0; j < nsteps; ++j) {
+            const int nsteps_all = SPARSE ? ctl->steps[2] : nkv;
+            auto issue_kv = [&](int j) {  // K/V tiles of step j into stage j % STAGES
                 const int kt = SPARSE ? ulist[j] : j;  // key tile of step j
                 const int s = j % C::STAGES;
-                if (j >= C::STAGES &&
-                    !wait_one(&ctl->kv_empty[s], ((j / C::STAGES) - 1) & 1, p.err, &ctl->abort, false, 1))
-                    break;
                 mbar_arrive_expect_tx(&ctl->kv_full[s], EXPORT_S ? C::K_BYTES : C::K_BYTES + C::V_BYTES);
                 tma_load_3d(sK + s * C::K_BYTES, &tm_k, &ctl->kv_full[s], 0, (kv0 + kt) * C::BN, bh);
                 if (!EXPORT_S)
                     tma_load_3d(sV + s * C::V_BYTES, &tm_v, &ctl->kv_full[s], 0, (kv0 + kt) * C::BN, bh);
                 issued = j + 1;
+            };
+            if (KRES) {
+                // the ring's first stage takes its K/V tiles at once
+                if (nsteps_all > 0) issue_kv(0);
+                // bf16 Q rows of both tiles into the ring's (still idle) stages 1
+                // and 2: tile t's [channel half][128 rows][64], 128-byte swizzle
+                const int b = bh / p.H, h = bh % p.H;
+                mbar_arrive_expect_tx(&ctl->qb_full, 2 * C::BM * D * 2);
+                for (int t = 0; t < 2; ++t)
+                    for (int half = 0; half < D / 64; ++half) {
+                        uint8_t *dst = sQb[t] + half * C::BM * 128;
+                        const int n = (qt0 + t) * C::BM;
+                        if (p.q_swap)
+                            tma_load_4d(dst, &tm_qb, &ctl->qb_full, half * 64, h, n, b);
+                        else
+                            tma_load_4d(dst, &tm_qb, &ctl->qb_full, half * 64, n, h, b);
+                    }
+                // the block means, a chunk at a time, into the (still idle) P
+                // buffers, each once the tensor core finished with the last
+                for (int c = 0; pro_ok && c < e_chunks; ++c) {
+                    if (c >= 1 && !(pro_ok = wait_one(&ctl->e_full[0], (c - 1) & 1, p.err, &ctl->abort, false, 1)))
+                        break;
+                    mbar_arrive_expect_tx(&ctl->mb_full[0], kEChunk * D * 2);
+                    for (int half = 0; half < D / 64; ++half)
+                        tma_load_3d(sP + half * kEChunk * 128, &tm_mean, &ctl->mb_full[0], half * 64, c * kEChunk, bh);
+                    m_issued = c + 1;
+                }
+                // the ring's stages 1 and 2 and the P buffers are free once the
+                // last products are done (the MMAs complete in order)
+                if (pro_ok && e_chunks > 0) pro_ok = wait_one(&ctl->e_full[0], (e_chunks - 1) & 1, p.err, &ctl->abort, false, 1);
+            }
+            const int nsteps = !pro_ok ? 0 : nsteps_all;
+            for (int j = issued; j < nsteps; ++j) {
+                if (j >= C::STAGES &&
+                    !wait_one(&ctl->kv_empty[j % C::STAGES], ((j / C::STAGES) - 1) & 1, p.err, &ctl->abort, false, 1))
+                    break;
+                issue_kv(j);
             }
             // every copy started here lands before the CTA may exit
             wait_one(FUSED_Q ? &ctl->qb_full : &ctl->q_full, 0, p.err, &ctl->abort, true, 2);
+            if (KRES) {
+                wait_one(&ctl->qb_full, 0, p.err, &ctl->abort, true, 2);
+                // each means chunk after the first went out after the previous one's
+                // products were done, so only the last one issued can be in flight
+                if (m_issued > 0) wait_one(&ctl->mb_full[0], (m_issued - 1) & 1, p.err, &ctl->abort, true, 2);
+            }
             for (int j = issued > C::STAGES ? issued - C::STAGES : 0; j < issued; ++j)
                 wait_one(&ctl->kv_full[j % C::STAGES], (j / C::STAGES) & 1, p.err, &ctl->abort, true, 3);
         }
@@ -478,8 +553,36 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 if (ok) tc_commit_if(me, &ctl->kv_empty[s]);
             }
         } else {
-        bool ok = wait_warp(&ctl->q_full, 0, p.err, &ctl->abort, 4) &&
-                  wait_warp(&ctl->kv_full[0], 0, p.err, &ctl->abort, 5);
+        bool ok = true;
+        if constexpr (KRES) {
+            // mean-term products: tile t's accumulator at columns [256 t, 256 t + N)
+            const uint64_t dqb[2] = {smem_desc_kmajor(smem_u32(sQb[0]), 128),   // [half][128][64] bf16
+                                     smem_desc_kmajor(smem_u32(sQb[1]), 128)};
+            const uint64_t dmb = smem_desc_kmajor(smem_u32(sP), 128);        // [half][256][64] bf16
+            ok = wait_warp(&ctl->qb_full, 0, p.err, &ctl->abort, 4);
+            for (int c = 0; ok && c < e_chunks; ++c) {
+                const int nb = min(kEChunk, p.nkb - c * kEChunk);
+                const uint32_t idesc = idesc_bf16_f32(128, (nb + 15) & ~15);
+                if (!(ok = wait_warp(&ctl->mb_full[0], c & 1, p.err, &ctl->abort, 5))) break;
+                // tensor memory held chunk c - 1: the softmax took it out
+                if (c >= 1 && !(ok = wait_warp(&ctl->e_free[0], (c - 1) & 1, p.err, &ctl->abort, 7))) break;
+                tc_fence_after();
+#pragma unroll
+                for (int t = 0; t < 2; ++t)
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        // K step kk: channels 16 kk.. = 32 bytes into the rows of half kk / 4
+                        const uint64_t a = dqb[t] + (uint64_t)((((kk / 4) * C::BM * 128) + (kk % 4) * 32) >> 4);
+                        const uint64_t bm = dmb + (uint64_t)((((kk / 4) * kEChunk * 128) + (kk % 4) * 32) >> 4);
+                        mma_f16_ss_if(me, tmem + t * 256, a, bm, idesc, kk > 0 ? 1u : 0u);
+                    }
+                tc_commit_if(me, &ctl->e_full[0]);
+            }
+            // tensor memory is the softmax warps' again before the first QK
+            if (ok && e_chunks > 0) ok = wait_warp(&ctl->e_free[0], (e_chunks - 1) & 1, p.err, &ctl->abort, 7);
+        }
+        ok = ok && wait_warp(&ctl->q_full, 0, p.err, &ctl->abort, 4) &&
+             wait_warp(&ctl->kv_full[0], 0, p.err, &ctl->abort, 5);
         if (ok) {
             tc_fence_after();
             issue_qk(0, 0);
@@ -577,6 +680,34 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         } else {
             sq = qt < p.nqb ? p.q_scale[(int64_t)bh * p.nqb + qt] : 0.f;
         }
+        float *eslot = nullptr;  // KRES: this CTA's scratch slot, [nkb][256 rows]
+        if constexpr (KRES) {
+            uint32_t smid;
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+            if (static_cast<int>(smid) >= p.n_slots) {
+                // no slot for this SM: give up (reported like a timed-out wait, site 0)
+                if (lane == 0) record_timeout(p.err, &ctl->abort, 0);
+                ok = false;
+            } else {
+                eslot = p.eslot + (int64_t)smid * p.nkb * 256 + t * 128 + row;
+            }
+            for (int c = 0; ok && c < e_chunks; ++c) {
+                if (!(ok = wait_warp(&ctl->e_full[0], c & 1, p.err, &ctl->abort, 14))) break;
+                tc_fence_after();
+                const int nb = min(kEChunk, p.nkb - c * kEChunk);
+                for (int cc = 0; cc < nb; cc += 32) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tmem + lane_off + t * 256 + cc, v);
+                    tmem_wait_ld_x32(v);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (cc + i < nb) eslot[(int64_t)(c * kEChunk + cc + i) * 256] = __uint_as_float(v[i]) * p.s_l2;
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->e_free[0]);
+            }
+        }
         const float cq = sq * p.s_l2;
         const float kLog2_448 = 8.807354922057604f;
         const float *ksc = p.k_scale + (int64_t)bh * p.nkb + 2 * kv0;
@@ -586,11 +717,9 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
         float m = -INFINITY, l = 0.f;
         float ks_next0 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next);
         float ks_next1 = (EXPORT_S || steps == 0) ? 0.f : __ldg(ksc + 2 * kt_next + 1);
-        // KRES: this row's mean terms, [K block][row] with a row stride of N_pad
-        const int64_t npad = (int64_t)p.nqb * C::BM;
-        const float *eb = KRES ? p.ebias + (int64_t)bh * p.nkb * npad + grow : nullptr;
-        float e_next0 = KRES ? __ldg(eb + (2 * kt_next) * npad) : 0.f;
-        float e_next1 = KRES ? __ldg(eb + (2 * kt_next + 1) * npad) : 0.f;
+        // KRES: this row's mean terms from the slot (written by this thread above)
+        float e_next0 = (KRES && ok) ? eslot[(2 * kt_next) * 256] : 0.f;
+        float e_next1 = (KRES && ok) ? eslot[(2 * kt_next + 1) * 256] : 0.f;
         for (int j = 0; ok && j < steps; ++j) {
             // this step's key tile and its two K-block scales were fetched one step ahead
             const int kt = kt_next;
@@ -601,8 +730,8 @@ __global__ void __launch_bounds__(Cfg<D>::THREADS, 1)
                 ks_next0 = __ldg(ksc + 2 * kt_next);
                 ks_next1 = __ldg(ksc + 2 * kt_next + 1);
                 if (KRES) {
-                    e_next0 = __ldg(eb + (2 * kt_next) * npad);
-                    e_next1 = __ldg(eb + (2 * kt_next + 1) * npad);
+                    e_next0 = eslot[(2 * kt_next) * 256];
+                    e_next1 = eslot[(2 * kt_next + 1) * 256];
                 }
             }
             if (!(ok = wait_warp(&ctl->s_full[t], j & 1, p.err, &ctl->abort, 10 + t))) break;
@@ -813,16 +942,24 @@ cudaError_t make_map(CUtensorMap *m, const void *base, uint64_t d0, uint64_t d1,
 
 template <int D, bool EXPORT_S, bool SPARSE, bool KRES = false, bool FUSED_Q = false>
 cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, const uint8_t *v_e4m3,
-                          const AttnParams &p0, dim3 grid, cudaStream_t st, const Src *q_bf16 = nullptr) {
+                          const AttnParams &p0, dim3 grid, cudaStream_t st, const Src *q_bf16 = nullptr,
+                          const uint16_t *k_bmean = nullptr) {
     using C = Cfg<D>;
     const int n_pad = s.n_pad();
-    CUtensorMap tq, tk, tv, tqb;
+    CUtensorMap tq, tk, tv, tqb, tmean;
     AttnParams p = p0;
     cudaError_t e;
     if (FUSED_Q) {
         if (!q_bf16) return cudaErrorInvalidValue;
         if ((e = make_bf16_token_map(&tqb, *q_bf16, s, 64, &p.q_swap)) != cudaSuccess) return e;
         q_i8 = k_i8;  // the INT8 Q map is not read; any valid map will do
+    }
+    if (KRES) {
+        // bf16 Q rows (128 per box, 128-byte swizzle) and the bf16 block means
+        // [BH][nkb][d] (256 blocks per box, 128-byte swizzle) for the prologue
+        if (!q_bf16 || !k_bmean) return cudaErrorInvalidValue;
+        if ((e = make_bf16_token_map(&tqb, *q_bf16, s, C::BM, &p.q_swap, true)) != cudaSuccess) return e;
+        if ((e = make_bf16_map3(&tmean, k_bmean, D, s.n_kblocks(), s.BH(), 256)) != cudaSuccess) return e;
     }
     if ((e = make_map(&tq, q_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BM)) != cudaSuccess) return e;
     if ((e = make_map(&tk, k_i8, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) return e;
@@ -831,7 +968,8 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     } else if ((e = make_map(&tv, v_e4m3, D, n_pad, s.BH(), D, (uint64_t)n_pad * D, D, C::BN)) != cudaSuccess) {
         return e;
     }
-    if (!FUSED_Q) tqb = tq;  // not read
+    if (!FUSED_Q && !KRES) tqb = tq;  // not read
+    if (!KRES) tmean = tq;              // not read
     p.err = device_error_ptr();
     if (!p.err) return cudaErrorSymbolNotFound;
     const int smem = smem_bytes<D>(SPARSE ? 7 * p.nqb + 8 : 0);  // three uint16 lists and one uint8 list
@@ -843,7 +981,7 @@ cudaError_t launch_attn_d(const Shape &s, const int8_t *q_i8, const int8_t *k_i8
     if ((e = cudaFuncGetAttributes(&fa, kern)) != cudaSuccess) return e;
     if (fa.numRegs != C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
     if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    return launch_dependent(kern, grid, dim3(C::THREADS), smem, st, tq, tk, tv, tqb, p);
+    return launch_dependent(kern, grid, dim3(C::THREADS), smem, st, tq, tk, tv, tqb, tmean, p);
 }
 
 }  // namespace
@@ -860,7 +998,8 @@ unsigned *device_error_ptr() {
     return ptrs[dev];
 }
 
-cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped) {
+cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped,
+                                bool swizzle128) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return cudaErrorSymbolNotFound;
     // Dimensions after the channels: N and H in order of stride, then B.  A
@@ -884,9 +1023,26 @@ cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, 
     const cuuint32_t box[4] = {64, swap ? 1u : rows, swap ? rows : 1u, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<uint16_t *>(src.p), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                    CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     *hn_swapped = swap ? 1 : 0;
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+// 3-D map of a contiguous bf16 [d2][d1][d0] array (d0 = 64 or 128 channels):
+// box 64 channels x `rows` x 1, 128-byte swizzle, zeros outside the array.
+cudaError_t make_bf16_map3(CUtensorMap *m, const uint16_t *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                           uint32_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return cudaErrorSymbolNotFound;
+    const cuuint64_t dims[3] = {d0, d1, d2};
+    const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    const cuuint32_t box[3] = {64, rows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
@@ -926,13 +1082,23 @@ cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &
                : launch_attn_d<64, false, false, false, true>(s, nullptr, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16);
 }
 
-cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,
-                                  cudaStream_t st) {
+int kres_slots() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess)
+        return 0;
+    return sms;
+}
+
+cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Src &q_bf16, const uint16_t *k_bmean,
+                                  const Dst &out, float sm_scale, float *eslot, int n_slots, cudaStream_t st) {
     AttnParams p = attn_params(s, c, out, sm_scale);
-    p.ebias = ebias;
+    p.eslot = eslot;
+    p.n_slots = n_slots;
     dim3 grid((s.n_qblocks() + 1) / 2, s.BH());
-    return s.d == 128 ? launch_attn_d<128, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st)
-                      : launch_attn_d<64, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st);
+    return s.d == 128
+               ? launch_attn_d<128, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16, k_bmean)
+               : launch_attn_d<64, false, false, true>(s, c.q_i8, c.k_i8, c.v_e4m3, p, grid, st, &q_bf16, k_bmean);
 }
 
 cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &out, float sm_scale,

@@ -263,6 +263,18 @@ __device__ __forceinline__ void mma_f8_ss_if(bool me, uint32_t d_tmem, uint64_t 
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(static_cast<uint32_t>(me))
         : "memory");
 }
+// D(tmem) (+)= A(smem) * B(smem)^T, 16-bit float inputs (bf16 or f16, both the
+// same, from idesc), fp32 accumulate.
+__device__ __forceinline__ void mma_f16_ss_if(bool me, uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                              uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "setp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(static_cast<uint32_t>(me))
+        : "memory");
+}
 __device__ __forceinline__ void tc_commit_if(bool me, uint64_t *bar) {
     asm volatile(
         "{\n\t.reg .pred q;\n\t"
@@ -309,6 +321,10 @@ __host__ __device__ constexpr uint32_t idesc_i8_s32(uint32_t M, uint32_t N) {
 }
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(uint32_t M, uint32_t N) {
     return (1u << 4) | (0u << 7) | (0u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
+}
+// kind::f16 with bf16 A and B (format 1 in both fields) and an fp32 D.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 // The same with an MN-major B operand (bit 16).
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32_bmn(uint32_t M, uint32_t N) {

@@ -93,7 +93,12 @@ cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *
 // 4-D tiled TMA map of a bf16 [B,H,N,d] view: box = 64 channels x `rows` tokens
 // of one (b,h).  The N and H dimensions are handed to the hardware in stride
 // order; *hn_swapped tells the kernel which coordinate comes second.
-cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped);
+cudaError_t make_bf16_token_map(CUtensorMap *m, const Src &src, const Shape &s, uint32_t rows, int *hn_swapped,
+                                bool swizzle128 = false);
+// 3-D tiled TMA map of a contiguous bf16 [d2][d1][d0] array: box 64 x rows x 1,
+// 128-byte swizzle, zeros outside the array.
+cudaError_t make_bf16_map3(CUtensorMap *m, const uint16_t *base, uint64_t d0, uint64_t d1, uint64_t d2,
+                           uint32_t rows);
 // Device error word (bounded waits that gave up) of the current device.
 unsigned *device_error_ptr();
 
@@ -126,15 +131,16 @@ cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &o
 // (c.q_i8 / c.q_scale are not used).
 cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &q_bf16, const Dst &out,
                                      float sm_scale, cudaStream_t st);
-// K-residual mode: attention with the mean term ebias [BH][nkb][N_pad] added
-// to the scores (sage_attn.cu); the residual codes and the mean term
-// (sage_kres.cu).
-cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Dst &out, float sm_scale, const float *ebias,
-                                  cudaStream_t st);
+// K-residual mode: the residual codes and bf16 block means (sage_kres.cu),
+// and the attention kernel that computes the mean term (q . mean_b) in its
+// prologue on the tensor cores from the bf16 Q rows and the block means,
+// keeping it in per-SM scratch slots of kres_slots() x nkb x 256 floats
+// (sage_attn.cu).  kres_slots() is the current device's SM count (0 on error).
 cudaError_t launch_kres(const Shape &s, const Src &k, int8_t *k_i8, float *k_scale, uint16_t *k_bmean,
                         cudaStream_t st);
-cudaError_t launch_ebias(const Shape &s, const Src &q, const uint16_t *k_bmean, float sm_scale, float *ebias,
-                         cudaStream_t st);
+int kres_slots();
+cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Src &q_bf16, const uint16_t *k_bmean,
+                                  const Dst &out, float sm_scale, float *eslot, int n_slots, cudaStream_t st);
 cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_t *k_i8, int bh, int q_tile,
                                  int kv_tile, int32_t *s_out, cudaStream_t st);
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st);
