@@ -97,12 +97,13 @@ sage_status_t sage_check(sage_stream_t stream);
  * 0 for an invalid shape.  Layout inside it is private. */
 size_t sage_attn_workspace_bytes(int B, int H, int N, int d);
 
-/* Bytes of scratch sage_quant_qk / sage_quant_v need (the per-chunk partial
- * statistics of the smoothing mean and of the V channel maxima): with
- * C = ceil(N/256) chunks and up(x) = x rounded up to 1024,
- *   up(8*B*H*C*d) + up(4*B*H*C*d) + 2*up(4*B*H*d)
- * (fp64 K sums and fp32 V maxima per chunk, then the fp32 K mean and V factor
- * per head); 0 for an invalid shape. */
+/* Bytes of scratch sage_quant_qk / sage_quant_v need (the partial statistics
+ * of the smoothing mean and of the V channel maxima, one per pair of a head
+ * and a CTA of the quantize kernel that covers part of it): with
+ * S = B*H + min(512, B*H*ceil(N/128)) slots and up(x) = x rounded up to 1024,
+ *   up(8*S*d) + up(4*S*d) + up(8*S)
+ * (fp64 K sums, fp32 V maxima and a 64-bit publication flag per slot); 0 for
+ * an invalid shape.  Nothing in it needs to start at zero. */
 size_t sage_quant_workspace_bytes(int B, int H, int N, int d);
 
 /*
@@ -139,12 +140,12 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4],
  *   workspace.  The statistics scratch is a fixed array of
  *   SAGE_NOALLOC_SCRATCH_BYTES (4 MiB) inside the library's device memory;
  *   every GPU that loads the library holds it until the process exits.  A shape
- *   whose scratch (sage_quant_workspace_bytes, about 12*B*H*d*ceil(N/256)
- *   bytes) exceeds it is rejected with SAGE_ERR_WORKSPACE before anything is
- *   launched: e.g. (1,24,4608,128) needs 0.69 MB and (1,24,16384,128) 2.4 MB
- *   and fit, (1,40,34020,128) needs 8.2 MB and (1,24,65536,128) 9.5 MB and do
- *   not.  The inputs must be on the current device (SAGE_ERR_INVALID_ARG
- *   otherwise).  The call allocates nothing.
+ *   whose scratch (sage_quant_workspace_bytes, about 12*d*(B*H + 512) bytes)
+ *   exceeds it is rejected with SAGE_ERR_WORKSPACE before anything is
+ *   launched: e.g. (1,24,4608,128) and (1,24,65536,128) need 0.83 MB and
+ *   (1,40,34020,128) 0.85 MB and fit; with d = 128 up to about 2200 heads
+ *   (B*H) fit, with d = 64 about 4900.  The inputs must be on the current
+ *   device (SAGE_ERR_INVALID_ARG otherwise).  The call allocates nothing.
  *   The first call on each device looks up the array's device address (with
  *   that device current) and keeps it; make that first call before any stream
  *   capture, and do not go on using the library after cudaDeviceReset.

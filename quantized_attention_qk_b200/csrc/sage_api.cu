@@ -120,24 +120,21 @@ void set_last_error(const char *fmt, ...) {
     g_last_error = buf;
 }
 
-// Statistics scratch: fp64 K column sums and fp32 V column maxima per
-// 256-token chunk, then the fp32 K mean and V factor per (b,h, channel).
+// Statistics scratch: per slot the fp64 K column sums, the fp32 V column
+// maxima and a 64-bit flag.
 size_t stats_ws_bytes(const Shape &s) {
-    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d;
-    const size_t per = (size_t)s.BH() * s.d * sizeof(float);
-    return up(part * sizeof(double)) + up(part * sizeof(float)) + 2 * up(per);
+    const size_t slots = static_cast<size_t>(s.stats_slots());
+    return up(slots * s.d * sizeof(double)) + up(slots * s.d * sizeof(float)) + up(slots * 8);
 }
 
 StatsWs carve_stats_ws(void *base, const Shape &s) {
     char *p = static_cast<char *>(base);
-    const size_t part = (size_t)s.BH() * s.n_chunks() * s.d;
-    const size_t kpart = up(part * sizeof(double)), vpart = up(part * sizeof(float));
-    const size_t per = up((size_t)s.BH() * s.d * sizeof(float));
+    const size_t slots = static_cast<size_t>(s.stats_slots());
+    const size_t kpart = up(slots * s.d * sizeof(double)), vpart = up(slots * s.d * sizeof(float));
     StatsWs w;
     w.ksum_part = reinterpret_cast<double *>(p);
     w.vmax_part = reinterpret_cast<float *>(p + kpart);
-    w.k_mean = reinterpret_cast<float *>(p + kpart + vpart);
-    w.v_inv = reinterpret_cast<float *>(p + kpart + vpart + per);
+    w.flags = reinterpret_cast<unsigned long long *>(p + kpart + vpart);
     return w;
 }
 
@@ -226,9 +223,8 @@ sage_status_t sage_quant_qk(const void *q_bf16, const int64_t q_stride[4], const
     c.q_scale = q_scale;
     c.k_i8 = k_i8;
     c.k_scale = k_scale;
-    cudaError_t e = launch_stats(s, &ks, nullptr, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, &ks, nullptr, ws, k_mean, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, &qs, &ks, nullptr, ws, k_mean, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     return SAGE_OK;
 }
 
@@ -249,9 +245,8 @@ sage_status_t sage_quant_v(const void *v_bf16, const int64_t v_stride[4], int B,
     Codes c{};
     c.v_e4m3 = v_e4m3;
     c.v_scale = v_scale;
-    cudaError_t e = launch_stats(s, nullptr, &vs, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, nullptr, nullptr, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, nullptr, nullptr, &vs, ws, nullptr, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     return SAGE_OK;
 }
 
@@ -302,9 +297,8 @@ sage_status_t sage_attn_fwd_ev(const void *q, const int64_t q_stride[4], const v
     const Codes c = carve_codes(scr.ptr, s);
     const StatsWs ws = carve_stats_ws(static_cast<char *>(scr.ptr) + cb, s);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, &qs, &ks, &vs, ws, nullptr, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_attention(s, c, dst(out, o_stride), sm_scale, st)) != cudaSuccess)
@@ -399,9 +393,8 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], con
     const Codes c = carve_codes(base, s);
     const StatsWs ws = carve_stats_ws(base + cb, s);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, &qs, &ks, &vs, ws, nullptr, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     // tau >= 1 keeps every key tile (reading S3): the dense kernel computes the
     // same result bit for bit without walking step lists
     const bool dense = !mask_in && tau >= 1.f;
@@ -445,9 +438,8 @@ sage_status_t sage_attn_fwd_fused_q(const void *q, const int64_t q_stride[4], co
     const Codes c = carve_codes(scr.ptr, s);
     const StatsWs ws = carve_stats_ws(static_cast<char *>(scr.ptr) + cb, s);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_stats(s, &ks, &vs, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, nullptr, &ks, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, nullptr, &ks, &vs, ws, nullptr, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_attention_fused_q(s, c, qs, dst(out, o_stride), sm_scale, st)) != cudaSuccess)
@@ -505,9 +497,8 @@ sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4], const
     uint16_t *bmean = reinterpret_cast<uint16_t *>(base + cb + sb);
     float *eslot = reinterpret_cast<float *>(base + cb + sb + mb);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_stats(s, nullptr, &vs, ws, st);
-    if (e != cudaSuccess) return cuda_fail(e, "statistics pass");
-    if ((e = launch_quant(s, &qs, nullptr, &vs, ws, nullptr, c, st)) != cudaSuccess) return cuda_fail(e, "quantize pass");
+    cudaError_t e = launch_qpass(s, &qs, nullptr, &vs, ws, nullptr, c, st);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     if ((e = launch_kres(s, ks, c.k_i8, c.k_scale, bmean, st)) != cudaSuccess)
         return cuda_fail(e, "K-residual quantization");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)

@@ -209,9 +209,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
             const Dst o{d_out + ooff, (int64_t)H * nd, nd, d};
             const Codes codes = carve_codes(ws, cs);
             const StatsWs sw = carve_stats_ws(ws + up(codes_bytes(cs)), cs);
-            if ((e = launch_stats(cs, &k, &v, sw, s)) != cudaSuccess)
-                return finish(SAGE_ERR_CUDA, e, "statistics pass");
-            if ((e = launch_quant(cs, &q, &k, &v, sw, nullptr, codes, s)) != cudaSuccess)
+            if ((e = launch_qpass(cs, &q, &k, &v, sw, nullptr, codes, s)) != cudaSuccess)
                 return finish(SAGE_ERR_CUDA, e, "quantize pass");
             if ((e = launch_attention(cs, codes, o, sm_scale, s)) != cudaSuccess)
                 return finish(SAGE_ERR_CUDA, e, "attention kernel");

@@ -16,7 +16,7 @@ namespace sage {
 constexpr int kQBlock = 128;       // Q tokens per quantization block == attention query tile
 constexpr int kKBlock = 64;        // K tokens per quantization block
 constexpr int kKvTile = 128;       // keys per attention KV tile (two K blocks)
-constexpr int kStatsRows = 256;    // statistics pass: tokens per chunk (a multiple of 64)
+constexpr int kStatsMaxGrid = 512;  // quantize pass: at most this many CTAs (bounds its statistics slots)
 constexpr unsigned kErrTimeoutBit = 1u;  // device error word: a bounded wait gave up
 constexpr int kMaxSelectTiles = 4096;    // block-sparse selection: key tiles one row ranks in shared memory
 
@@ -36,27 +36,26 @@ struct Shape {
     int n_pad() const { return ((N + kQBlock - 1) / kQBlock) * kQBlock; }
     int n_qblocks() const { return n_pad() / kQBlock; }
     int n_kblocks() const { return n_pad() / kKBlock; }
-    // Statistics pass: each (b,h) is cut into n_chunks() token chunks of
-    // chunk_rows() rows.  The size depends on nothing but itself, so the fp32
-    // sums (and hence the codes) of a head do not depend on which other heads
-    // share the call.
-    int chunk_rows() const { return kStatsRows; }
-    int n_chunks() const { return (N + chunk_rows() - 1) / chunk_rows(); }
+    // Quantize pass: one statistics partial per (CTA, head) it covers, kept in
+    // slot CTA + head: at most BH + min(kStatsMaxGrid, 128-token blocks) slots.
+    long long stats_slots() const {
+        const long long blocks = (long long)BH() * n_qblocks();
+        return BH() + (blocks < kStatsMaxGrid ? blocks : kStatsMaxGrid);
+    }
     // Block-sparse masks: one row of mask_words() 32-bit words per (b,h, query
     // tile), bit j = key tile j (tiles of kKvTile tokens for both).
     int n_tiles() const { return (N + kKvTile - 1) / kKvTile; }
     int mask_words() const { return (n_tiles() + 31) / 32; }
 };
 
-// Scratch of the quantize pass: per-chunk partials and the finished statistics.
+// Scratch of the quantize pass: the statistics partials and their flags.
 // The K column sums are fp64: a sum of bf16 values is exact there whenever the
 // column's values span fewer than 53 bits (every workload here), so the mean
 // does not depend on the order of the additions.
 struct StatsWs {
-    double *ksum_part;  // [BH][chunks][d]
-    float *vmax_part;  // [BH][chunks][d]
-    float *k_mean;     // [BH][d]
-    float *v_inv;      // [BH][d]  448 / amax (0 for an all-zero channel)
+    double *ksum_part;          // [slots][d]
+    float *vmax_part;           // [slots][d]
+    unsigned long long *flags;  // [slots]
 };
 
 // Codes and scales consumed by the attention kernel.
@@ -84,11 +83,11 @@ StatsWs carve_stats_ws(void *base, const Shape &s);
 size_t codes_bytes(const Shape &s);
 Codes carve_codes(void *base, const Shape &s);
 
-// Quantize pass launchers (sage_quant.cu): per-chunk partial statistics of K
-// and V, then the codes (the statistics are finished inside the second kernel).
-// `user_k_mean` may be null; the V scales go to c.v_scale.
-cudaError_t launch_stats(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, cudaStream_t st);
-cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
+// The quantize pass (sage_quant.cu) in one cooperatively launched kernel:
+// statistics of k and/or v, then the codes of the tensors given (null ones are
+// skipped; the combinations q+k+v, q+k, k+v, v and q+v).  `user_k_mean` may be
+// null; the V scales go to c.v_scale.
+cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
                          float *user_k_mean, const Codes &c, cudaStream_t st);
 // 4-D tiled TMA map of a bf16 [B,H,N,d] view: box = 64 channels x `rows` tokens
 // of one (b,h).  The N and H dimensions are handed to the hardware in stride

@@ -1,26 +1,42 @@
 // sage_quant.cu -- the quantize pass of the quantized attention forward.
 //
-// Two HBM-bound streaming kernels (no tensor cores: there is no contraction):
-//   k_stats  per (b,h, token chunk): sum of K (fp64, exact for bf16 inputs
-//            whose values span fewer than 53 bits) and max |V| per channel
-//            over the chunk, 64-token blocks staged through a 3-deep TMA ring
-//   k_quant  per (b,h, 128-token block): finishes this (b,h)'s statistics from
-//            the chunk partials (the K mean, the smoothing statistic, and the
-//            448/amax factors of V) while TMA brings the block's Q, K and V
-//            rows into shared memory, then Q block -> INT8, (K - mean) per
-//            64-token block -> INT8, V -> e4m3 (token-major, like the codes of
-//            Q and K; the attention kernel reads it as an MN-major operand).
 // Pages: "MiniMax H3 接入 SageAttention 实测加速", section 一 (outlier smoothing of
 // QK^T, INT8 QK, FP8 PV).  Block sizes, rounding and scale conventions are the
 // readings C1-C3 and C7 of the design notes:
 //   scale = amax/127 (fp32 IEEE divide), code = rne(x * fp32(127/amax)) in
 //   [-127,127]; V: code = e4m3_rn_satfinite(v * fp32(448/amax_c)).
-// Inputs are read through 4-D tensor maps over arbitrary (b,h,n) strides, so a
-// fused-qkv view is read in place; codes are stored as 8-byte vectors.
+//
+// One HBM-bound streaming kernel, k_qpass (no tensor cores: there is no
+// contraction), launched cooperatively so that all its CTAs are resident at
+// once, in two phases:
+//   A  statistics: CTA i takes the i-th of G equal parts of all (b,h, 64-token
+//      sub-block)s; within each head its part covers, the warps stream the
+//      K and V rows (direct 16-byte loads held in registers, kept in L2 for
+//      phase B) and accumulate per channel the fp64 sum of K and the max |V|;
+//      the warps' results are added in warp order into one partial per
+//      (CTA, head), published with a release store of a flag.
+//   B  codes: CTA i takes the i-th of G equal parts of the (b,h, 128-token
+//      block)s -- the same part of the token range, last block first, so the
+//      K and V rows read most recently in phase A are the first ones reused.
+//      For each head it waits (acquire loads, bounded) for the flags of the
+//      CTAs that covered the head in phase A, adds their partials in CTA
+//      order (fp64) and finishes the statistics (the K mean and the 448/amax
+//      factors of V).  Then each 128-token block is coded from registers by
+//      a group of warps (16 rows each for d = 128, 32 for d = 64): Q block
+//      -> INT8 (the group exchanges its warps' maxima through shared memory),
+//      (K - mean) per 64-token block -> INT8, V -> e4m3 (token-major, like
+//      the codes of Q and K; the attention kernel reads it as an MN-major
+//      operand).
+// Warps work on their own rows and exchange block maxima only within their
+// group; the only CTA-wide barriers are at head boundaries.  The fp64 K sums are exact for bf16 inputs whenever a column's
+// values span fewer than 53 bits, so the mean does not depend on how the rows
+// were split among CTAs and warps.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
+#include <chrono>
 
 #include "sage_device.cuh"
 #include "sage_internal.h"
@@ -28,535 +44,447 @@
 namespace sage {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kPassWarps = 16;
+constexpr int kPassThreads = 32 * kPassWarps;
 
-__device__ __forceinline__ float warp_max(float v) {
+// Geometry of one warp's rows for head dim D: a warp load instruction covers
+// RPI rows of VPR 16-byte vectors; a lane holds NB vectors of each of Q, K and
+// V in phase B (RB rows per warp) and NA of K and of V in phase A (RA rows); a
+// 128-token block takes a group of WU warps, a 64-token K block KW of them.
+template <int D>
+struct Geom {
+    static constexpr int VPR = D / 8;
+    static constexpr int RPI = 32 / VPR;
+    static constexpr int NB = 8;
+    static constexpr int RB = NB * RPI;
+    static constexpr int WU = kQBlock / RB;
+    static constexpr int KW = kKBlock / RB;
+    static constexpr int GROUPS = kPassWarps / WU;
+    static constexpr int NA = 8;
+    static constexpr int RA = NA * RPI;
+};
+static_assert(Geom<128>::WU * Geom<128>::RB == kQBlock && Geom<64>::WU * Geom<64>::RB == kQBlock &&
+                  Geom<128>::KW >= 1 && Geom<64>::KW >= 1 && kPassWarps % Geom<128>::WU == 0,
+              "a warp group codes a 128-token block; a K block spans whole warps");
+static_assert(kKBlock % Geom<128>::RA == 0 && kKBlock % Geom<64>::RA == 0, "phase-A batches tile a sub-block");
+static_assert(Geom<64>::GROUPS < 16, "named barriers 1..GROUPS");
+
+// 16 bytes of a read-only input, not kept in L1, with an L2 eviction policy.
+// The memory clobber keeps a block's loads after the previous block's stores,
+// so that no more than one block's rows are live in registers.
+__device__ __forceinline__ uint4 ld_in(const uint16_t *p, uint64_t policy) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p), "l"(policy)
+                 : "memory");
+    return r;
+}
+
+// Per-half max of |x| over bf16 pairs: max of the accumulated magnitudes and
+// the magnitudes of x (a NaN half is ignored, like fmaxf does).
+__device__ __forceinline__ uint32_t bmax_abs(uint32_t m, uint32_t x) {
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(x & 0x7fff7fffu));
+    return d;
+}
+__device__ __forceinline__ float bf_bits(uint32_t h) { return __uint_as_float(h << 16); }
+
+__device__ __forceinline__ void st_release_u64(unsigned long long *p, unsigned long long v) {
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long *p) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+// Barrier of the `threads` threads of warp group `id` (ids from 1; 0 is
+// __syncthreads').
+__device__ __forceinline__ void group_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Two e4m3 codes (round to nearest even, saturating to +-448): lo in the low
+// byte (cvt packs its first source in the high byte).
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .b16 t;\n\tcvt.rn.satfinite.e4m3x2.f32 t, %1, %2;\n\tcvt.u32.u16 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float warp_fmax(float v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
     return v;
 }
 
-constexpr int kRowsPerLoad = 64;   // tokens per TMA box
-constexpr int kStatsStages = 3;
-
-// Shared-memory tile of `rows` tokens of one (b,h): [d/64][rows][64] bf16, as
-// the 64-channel TMA boxes land.  Element (row, 8-channel vector cv) starts at:
-__device__ __forceinline__ int tile_off(int rows, int row, int cv) {
-    return ((cv >> 3) * rows + row) * 64 + (cv & 7) * 8;
-}
-__device__ __forceinline__ uint4 ld_tile(const uint16_t *tile, int off) {
-    return *reinterpret_cast<const uint4 *>(tile + off);
-}
-
-// Issue the TMA loads of `rows` (a multiple of 64) tokens from token n of (b,h)
-// into `tile` ([d/64][rows][64]), completing on `bar`.
-// `policy` is the L2 eviction policy of the rows.
-template <int D>
-__device__ __forceinline__ void load_rows(uint16_t *tile, int rows, const CUtensorMap *map, int swap, uint64_t *bar,
-                                          int n, int h, int b, uint64_t policy) {
+// x[i] = the 16 bytes at row row0 + i * RPI (stride sn elements from p), or
+// zeros for rows >= limit.  Rows are stepped through with one pointer, and the
+// common case of all rows valid takes no per-row test.
+template <int NV, int RPI>
+__device__ __forceinline__ void load_rows(uint4 (&x)[NV], const uint16_t *p, int64_t sn, int row0, int limit,
+                                          uint64_t policy) {
+    const uint16_t *r = p + (int64_t)row0 * sn;
+    const int64_t step = (int64_t)RPI * sn;
+    if (row0 + (NV - 1) * RPI < limit) {
 #pragma unroll
-    for (int half = 0; half < D / 64; ++half)
-        for (int r = 0; r < rows; r += kRowsPerLoad) {
-            uint16_t *dst = tile + (half * rows + r) * 64;
-            if (swap)
-                tma_load_4d_hint(dst, map, bar, half * 64, h, n + r, b, policy);
-            else
-                tma_load_4d_hint(dst, map, bar, half * 64, n + r, h, b, policy);
-        }
-}
-
-// Max over the block of three values at once (all threads get the results).
-// `sh` holds two slot sets [2][3][NT/32], used alternately (`set`): a set is
-// written again only by the call after next, which every thread reaches after
-// the next call's barrier, i.e. after all threads have read this call's slots;
-// so one barrier per call suffices.
-template <int NT>
-__device__ __forceinline__ void block_max3_n(float &a, float &b, float &c, float *shs, int set) {
-    constexpr int NW = NT / 32;
-    float *sh = shs + set * 3 * NW;
-    a = warp_max(a);
-    b = warp_max(b);
-    c = warp_max(c);
-    const int w = threadIdx.x >> 5;
-    if ((threadIdx.x & 31) == 0) { sh[w] = a; sh[NW + w] = b; sh[2 * NW + w] = c; }
-    __syncthreads();
-    a = sh[0];
-    b = sh[NW];
-    c = sh[2 * NW];
+        for (int i = 0; i < NV; ++i, r += step) x[i] = ld_in(r, policy);
+    } else {
 #pragma unroll
-    for (int i = 1; i < NW; ++i) { a = fmaxf(a, sh[i]); b = fmaxf(b, sh[NW + i]); c = fmaxf(c, sh[2 * NW + i]); }
-}
-
-// Persistent CTAs over the (b,h, token chunk) items, a contiguous range each,
-// with a ring of kStatsStages 64-token stages kept full across item boundaries.
-struct StatsArgs {
-    int H, BH, N, nch, chunk, per;  // per: items per CTA
-    int do_k, do_v, k_swap, v_swap;
-    double *ksum_part;  // [BH][nch][D]
-    float *vmax_part;   // [BH][nch][D]
-    unsigned *err;
-};
-
-template <int D>
-__global__ void __launch_bounds__(kThreads) k_stats(const __grid_constant__ CUtensorMap tk,
-                                                    const __grid_constant__ CUtensorMap tv, const StatsArgs a) {
-    constexpr int VPR = D / 8;              // 16-byte vectors per token row
-    constexpr int RPI = kThreads / VPR;     // rows covered per pass of the block
-    constexpr int TILE = kRowsPerLoad * D;  // elements of one tensor in one stage
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    uint16_t *ring = reinterpret_cast<uint16_t *>(smem_raw);                    // [stage][K,V][TILE]
-    double *red_s = reinterpret_cast<double *>(ring + kStatsStages * 2 * TILE);  // [warps][D]
-    float *red_m = reinterpret_cast<float *>(red_s + (kThreads / 32) * D);      // [RPI][D]
-    __shared__ uint64_t full[kStatsStages];
-    __shared__ AbortState abort_st;
-    __shared__ int bad;
-    const int n_items = a.nch * a.BH;
-    const int i0 = blockIdx.x * a.per, i1 = min(n_items, i0 + a.per);
-    const int cv = threadIdx.x % VPR, r0 = threadIdx.x / VPR;
-    const uint32_t bytes = (a.do_k + a.do_v) * TILE * 2;
-    grid_dep_launch();  // the quantize kernel may take each SM this CTA leaves
-    auto rows_of = [&](int item) {
-        const int n0 = (item % a.nch) * a.chunk;
-        return min(a.N, n0 + a.chunk) - n0;
-    };
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < kStatsStages; ++i) mbar_init(&full[i], 1);
-        abort_st.flag = 0;
-        bad = 0;
-        fence_barrier_init();
-    }
-    __syncthreads();
-    // Stage sequence numbers count the CTA's 64-token loads in order.  Thread 0
-    // keeps the producer state: the next sub-block to load, how many loads it
-    // issued, how many the block consumed, and how many it saw complete.
-    int p_item = i0, p_sb = 0, issued = 0, consumed = 0, waited = 0;
-    // K and V are read again by the quantize pass right after: keep them in L2
-    const uint64_t keep = l2_policy_evict_last();
-    auto issue_more = [&]() {
-        while (!bad && p_item < i1 && issued < consumed + kStatsStages) {
-            const int st = issued % kStatsStages;
-            uint16_t *base = ring + st * 2 * TILE;
-            const int bh = p_item / a.nch, b = bh / a.H, h = bh % a.H;
-            const int n = (p_item % a.nch) * a.chunk + p_sb * kRowsPerLoad;
-            mbar_arrive_expect_tx(&full[st], bytes);
-            if (a.do_k) load_rows<D>(base, kRowsPerLoad, &tk, a.k_swap, &full[st], n, h, b, keep);
-            if (a.do_v) load_rows<D>(base + TILE, kRowsPerLoad, &tv, a.v_swap, &full[st], n, h, b, keep);
-            ++issued;
-            if (++p_sb * kRowsPerLoad >= rows_of(p_item)) {
-                ++p_item;
-                p_sb = 0;
-            }
-        }
-    };
-    if (threadIdx.x == 0) issue_more();
-    int qbase = 0;  // sequence number of the item's first sub-block (every thread)
-    for (int item = i0; item < i1; ++item) {
-        const int rows = rows_of(item);
-        const int nsub = (rows + kRowsPerLoad - 1) / kRowsPerLoad;
-        double s[8];
-        float m[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) { s[e] = 0.0; m[e] = 0.f; }
-        for (int sb = 0; sb < nsub; ++sb) {
-            const int q = qbase + sb;
-            const int st = q % kStatsStages;
-            if (threadIdx.x == 0 && !bad) {
-                if (wait_one(&full[st], (q / kStatsStages) & 1, a.err, &abort_st, false, 0))
-                    waited = q + 1;
-                else
-                    bad = 1;
-            }
-            __syncthreads();
-            if (!bad) {
-                const uint16_t *kt = ring + st * 2 * TILE, *vt = kt + TILE;
-#pragma unroll
-                for (int i = 0; i < kRowsPerLoad / RPI; ++i) {
-                    const int row = r0 + i * RPI;
-                    if (sb * kRowsPerLoad + row < rows) {  // the box may reach into the next chunk
-                        float f[8];
-                        if (a.do_k) {
-                            unpack8(ld_tile(kt, tile_off(kRowsPerLoad, row, cv)), f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) s[e] = __dadd_rn(s[e], static_cast<double>(f[e]));
-                        }
-                        if (a.do_v) {
-                            unpack8(ld_tile(vt, tile_off(kRowsPerLoad, row, cv)), f);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) m[e] = fmaxf(m[e], fabsf(f[e]));
-                        }
-                    }
-                }
-            }
-            __syncthreads();  // the stage is free again
-            if (threadIdx.x == 0) {
-                consumed = q + 1;
-                issue_more();
-            }
-        }
-        qbase += nsub;
-        // the item's partials: the K sums of a warp's rows by shuffles (the
-        // lanes VPR apart hold the same channels), then the warps in order;
-        // the V maxima per row of the block, then per channel
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-#pragma unroll
-            for (int o = VPR; o < 32; o <<= 1) s[e] = __dadd_rn(s[e], __shfl_xor_sync(0xffffffffu, s[e], o));
-            red_m[r0 * D + cv * 8 + e] = m[e];
-        }
-        if ((threadIdx.x & 31) < VPR) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) red_s[(threadIdx.x >> 5) * D + cv * 8 + e] = s[e];
-        }
-        __syncthreads();
-        for (int c = threadIdx.x; c < D; c += kThreads) {
-            double ss = 0.0;
-            float mm = 0.f;
-            for (int w = 0; w < kThreads / 32; ++w) ss = __dadd_rn(ss, red_s[w * D + c]);
-            for (int r = 0; r < RPI; ++r) mm = fmaxf(mm, red_m[r * D + c]);
-            const int64_t o = (int64_t)item * D + c;  // item = bh * nch + chunk
-            if (a.do_k) a.ksum_part[o] = ss;
-            if (a.do_v) a.vmax_part[o] = mm;
-        }
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        // every copy started here lands before the CTA exits
-        for (int q = waited; q < issued; ++q)
-            wait_one(&full[q % kStatsStages], (q / kStatsStages) & 1, a.err, &abort_st, true, 0);
+        for (int i = 0; i < NV; ++i, r += step)
+            x[i] = row0 + i * RPI < limit ? ld_in(r, policy) : make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
-// Threads of a quantize CTA: 512 (one CTA per SM) for d = 128, 256 (two CTAs
-// per SM, so two items are in flight per SM) for d = 64.
-template <int D>
-__host__ __device__ constexpr int quant_threads() { return D == 128 ? 512 : 256; }
-
-// Persistent CTAs over the (b,h, 128-token block) items, a contiguous range
-// each (so consecutive items share a (b,h) and its statistics), two buffers:
-// the next item's Q, K and V rows land while the current one is coded.
-struct QuantArgs {
-    int H, BH, N, n_pad, nch, per;
-    int q_swap, k_swap, v_swap;
-    const double *ksum_part;  // [BH][nch][D]
-    const float *vmax_part;   // [BH][nch][D]
-    float *ws_k_mean, *ws_v_inv;         // [BH][D], written with the first block of each (b,h)
-    float *user_k_mean;                  // optional copy of the K mean
+// A flag of phase A holds (stamp << 16) | readers: the call's 48-bit stamp
+// and the number of phase-B CTAs that read the head (known from the split).
+// Each reader takes one off after its wait and the last one clears the flag,
+// so every flag is zero again when the kernel ends: a replay of the same
+// launch (a captured graph: same stamp) never finds its own stamp left over,
+// and a fresh workspace holds a given 48-bit stamp only by chance.
+struct PassArgs {
+    Src q, k, v;
+    int H, BH, N, n_pad;
+    double *ksum_part;          // [slots][D]: slot = CTA + head
+    float *vmax_part;           // [slots][D]
+    unsigned long long *flags;  // [slots]
+    unsigned long long stamp;   // 48 bits, bit 47 set
+    float *user_k_mean;         // optional copy of the K mean [BH][D]
     Codes c;
     unsigned *err;
 };
 
 template <int D, bool DO_Q, bool DO_K, bool DO_V>
-__global__ void __launch_bounds__(quant_threads<D>(), 512 / quant_threads<D>()) k_quant(const __grid_constant__ CUtensorMap tq,
-                                                        const __grid_constant__ CUtensorMap tk,
-                                                        const __grid_constant__ CUtensorMap tv, const QuantArgs a) {
-    constexpr int NTH = quant_threads<D>();
-    constexpr int VPR = D / 8;
-    constexpr int RPI = NTH / VPR;
-    constexpr int NI = kQBlock / RPI;  // vectors per thread in one 128-token block
-    constexpr int TILE = kQBlock * D;
-    constexpr int NT = (DO_Q ? 1 : 0) + (DO_K ? 1 : 0) + (DO_V ? 1 : 0);
-    constexpr int OQ = 0, OK = (DO_Q ? 1 : 0), OV = OK + (DO_K ? 1 : 0);  // tensor slots in a buffer
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    uint16_t *bufs = reinterpret_cast<uint16_t *>(smem_raw);  // [2][NT][TILE]
-    __shared__ uint64_t bar[2];
-    __shared__ float mu[D], vinv[D], vmax[D];
-    __shared__ float red[2 * 3 * (NTH / 32)];
+__global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
+    using Gm = Geom<D>;
+    constexpr int VPR = Gm::VPR, RPI = Gm::RPI, NB = Gm::NB, RB = Gm::RB, WU = Gm::WU, KW = Gm::KW, NA = Gm::NA,
+                  RA = Gm::RA;
+    constexpr int NW = kPassWarps;
+    constexpr bool STATS = DO_K || DO_V;
+    __shared__ double red_s[NW][D];
+    __shared__ float red_m[NW][D];
+    __shared__ float mu[D], vinv[D];
+    __shared__ float grp_max[Gm::GROUPS][2][2][WU];  // [group][unit parity][Q, K][warp]
     __shared__ AbortState abort_st;
     __shared__ int bad;
-    const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock;
-    const int n_items = nqb * a.BH;
-    const int i0 = blockIdx.x * a.per, i1 = min(n_items, i0 + a.per);
-    const int cv = threadIdx.x % VPR, r0 = threadIdx.x / VPR;
-
+    const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock, nsb = (a.N + kKBlock - 1) / kKBlock;
+    const int G = gridDim.x;  // <= the 128-token blocks, so every CTA codes at least one
+    const long long nA = (long long)a.BH * nsb, nB = (long long)a.BH * nqb;
+    // the CTA whose part holds unit x, of n units split in G equal parts
+    auto owner = [&](long long x, long long n) { return (int)(((x + 1) * G - 1) / n); };
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int vec = lane % VPR, rl = lane / VPR;  // this lane's 8 channels and row within a load
     if (threadIdx.x == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
         abort_st.flag = 0;
         bad = 0;
-        fence_barrier_init();
     }
     __syncthreads();
-    // the last reads of Q, K and V: let them leave L2 first
-    const uint64_t drop = l2_policy_evict_first();
-    auto issue = [&](int item, int buf) {
-        const int bh = item / nqb, blk = item % nqb, b = bh / a.H, h = bh % a.H;
-        uint16_t *base = bufs + buf * NT * TILE;
-        mbar_arrive_expect_tx(&bar[buf], NT * TILE * 2);
-        if (DO_Q) load_rows<D>(base + OQ * TILE, kQBlock, &tq, a.q_swap, &bar[buf], blk * kQBlock, h, b, drop);
-        if (DO_K) load_rows<D>(base + OK * TILE, kQBlock, &tk, a.k_swap, &bar[buf], blk * kQBlock, h, b, drop);
-        if (DO_V) load_rows<D>(base + OV * TILE, kQBlock, &tv, a.v_swap, &bar[buf], blk * kQBlock, h, b, drop);
-    };
-    int issued = 0, waited = 0;  // thread 0: loads issued, and seen complete
     grid_dep_launch();  // the attention kernel may take each SM this CTA leaves
-    // The rows are the caller's inputs, complete before the statistics kernel
-    // started: the first item's loads go out before the wait for that kernel's
-    // partials (and before anything here is written).
-    if (threadIdx.x == 0 && i0 < i1) {
-        issue(i0, 0);
-        issued = 1;
+
+    // ------------------------------------------------------------ phase A
+    if constexpr (STATS) {
+        const uint64_t keep = l2_policy_evict_last();  // phase B reads K and V again
+        const long long a0 = nA * blockIdx.x / G, a1 = nA * (blockIdx.x + 1) / G;
+        for (int h = (int)(a0 / nsb); h <= (int)((a1 - 1) / nsb); ++h) {
+            const long long s0 = a0 > (long long)h * nsb ? a0 : (long long)h * nsb;
+            const long long s1 = a1 < (long long)(h + 1) * nsb ? a1 : (long long)(h + 1) * nsb;
+            const int r_begin = (int)(s0 - (long long)h * nsb) * kKBlock;
+            const int r_end = min(a.N, (int)(s1 - (long long)h * nsb) * kKBlock);
+            const int nbat = (r_end - r_begin + RA - 1) / RA;
+            const int b = h / a.H, hh = h % a.H;
+            const uint16_t *kp = a.k.p + b * a.k.sb + hh * a.k.sh + vec * 8;
+            const uint16_t *vp = a.v.p + b * a.v.sb + hh * a.v.sh + vec * 8;
+            double s8[8];
+            uint32_t m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s8[e] = 0.0;
+            for (int bt = warp; bt < nbat; bt += NW) {
+                const int rb = r_begin + bt * RA + rl;
+                uint4 kx[DO_K ? NA : 1], vx[DO_V ? NA : 1];
+                if constexpr (DO_K) load_rows<NA, RPI>(kx, kp, a.k.sn, rb, r_end, keep);
+                if constexpr (DO_V) load_rows<NA, RPI>(vx, vp, a.v.sn, rb, r_end, keep);
+#pragma unroll
+                for (int i = 0; i < NA; ++i) {
+                    if (DO_K) {
+                        float f[8];
+                        unpack8(kx[i], f);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s8[e] = __dadd_rn(s8[e], static_cast<double>(f[e]));
+                    }
+                    if (DO_V) {
+                        m4[0] = bmax_abs(m4[0], vx[i].x);
+                        m4[1] = bmax_abs(m4[1], vx[i].y);
+                        m4[2] = bmax_abs(m4[2], vx[i].z);
+                        m4[3] = bmax_abs(m4[3], vx[i].w);
+                    }
+                }
+            }
+            // the lanes VPR apart hold the same channels, then the warps in order
+#pragma unroll
+            for (int o = VPR; o < 32; o <<= 1) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) s8[e] = __dadd_rn(s8[e], __shfl_xor_sync(0xffffffffu, s8[e], o));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) m4[j] = bmax_abs(m4[j], __shfl_xor_sync(0xffffffffu, m4[j], o));
+            }
+            if (lane < VPR) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) red_s[warp][vec * 8 + e] = s8[e];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    red_m[warp][vec * 8 + 2 * j] = bf_bits(m4[j] & 0xffffu);
+                    red_m[warp][vec * 8 + 2 * j + 1] = bf_bits(m4[j] >> 16);
+                }
+            }
+            __syncthreads();
+            const int slot = blockIdx.x + h;
+            for (int c = threadIdx.x; c < D; c += kPassThreads) {
+                double ss = 0.0;
+                float mm = 0.f;
+#pragma unroll
+                for (int w = 0; w < NW; ++w) {
+                    ss = __dadd_rn(ss, red_s[w][c]);
+                    mm = fmaxf(mm, red_m[w][c]);
+                }
+                if (DO_K) a.ksum_part[(int64_t)slot * D + c] = ss;
+                if (DO_V) a.vmax_part[(int64_t)slot * D + c] = mm;
+            }
+            __syncthreads();  // every partial is written (and red_* free again)
+            if (threadIdx.x == 0) {
+                const long long x0 = (long long)h * nqb;
+                const unsigned long long readers = owner(x0 + nqb - 1, nB) - owner(x0, nB) + 1;
+                st_release_u64(a.flags + slot, (a.stamp << 16) | readers);
+            }
+        }
     }
-    grid_dep_wait();
-    int cur_bh = -1;
-    for (int item = i0, k = 0; item < i1; ++item, ++k) {
-        const int buf = k & 1;
-        const int bh = item / nqb, blk = item % nqb;
-        if ((DO_K || DO_V) && bh != cur_bh) {
-            // this (b,h)'s statistics from the chunk partials, in chunk order:
-            // mean = fp32(fp64 sum / N) (IEEE divide, then one rounding to
-            // fp32), V factor 448 / amax
-            __syncthreads();  // every thread is done coding with the previous head's
-            for (int c = threadIdx.x; c < D; c += NTH) {
+
+    // ------------------------------------------------------------ phase B
+    const uint64_t drop = l2_policy_evict_first();  // the last reads of Q, K and V
+    const long long b0 = nB * blockIdx.x / G, b1 = nB * (blockIdx.x + 1) / G;
+    const int grp = warp / WU, gw = warp % WU;  // warp group (one 128-token block at a time) and place in it
+    int parity = 0;
+    for (int h = (int)((b1 - 1) / nqb); h >= (int)(b0 / nqb); --h) {
+        const int c0 = (int)((b0 > (long long)h * nqb ? b0 : (long long)h * nqb) - (long long)h * nqb);
+        const int c1 = (int)((b1 < (long long)(h + 1) * nqb ? b1 : (long long)(h + 1) * nqb) - (long long)h * nqb);
+        if constexpr (STATS) {
+            __syncthreads();  // every warp is done with the previous head's statistics
+            const int i0 = owner((long long)h * nsb, nA), i1 = owner((long long)h * nsb + nsb - 1, nA);
+            for (int t = threadIdx.x; t <= i1 - i0; t += kPassThreads) {
+                unsigned long long *f = a.flags + i0 + t + h;
+                const long long t0 = clock64();
+                bool ok = true;
+                while ((ld_acquire_u64(f) >> 16) != a.stamp) {
+                    if (*reinterpret_cast<volatile int *>(&abort_st.flag) || clock64() - t0 > kWaitLimitClocks) {
+                        if (!*reinterpret_cast<volatile int *>(&abort_st.flag)) record_timeout(a.err, &abort_st, 10);
+                        bad = 1;
+                        ok = false;
+                        break;
+                    }
+                    __nanosleep(64);
+                }
+                if (!ok) break;
+                // one reader fewer; the last clears the flag (the partials are
+                // written again only by a later launch)
+                if ((atomicAdd(f, ~0ull) & 0xffffull) == 1ull) atomicExch(f, 0ull);
+            }
+            __syncthreads();
+            if (bad) break;
+            // the head's statistics: partials in CTA order (written by other
+            // CTAs of this kernel: read through L2); mean = fp32(fp64 sum / N),
+            // V factor 448 / amax
+            for (int c = threadIdx.x; c < D; c += kPassThreads) {
                 double sum = 0.0;
                 float mx = 0.f;
-#pragma unroll 8
-                for (int ch = 0; ch < a.nch; ++ch) {
-                    const int64_t o = ((int64_t)bh * a.nch + ch) * D + c;
-                    if (DO_K) sum = __dadd_rn(sum, a.ksum_part[o]);
-                    if (DO_V) mx = fmaxf(mx, a.vmax_part[o]);
+                for (int i = i0; i <= i1; ++i) {
+                    const int64_t o = (int64_t)(i + h) * D + c;
+                    if (DO_K) sum = __dadd_rn(sum, __ldcg(a.ksum_part + o));
+                    if (DO_V) mx = fmaxf(mx, __ldcg(a.vmax_part + o));
                 }
-                mu[c] = __double2float_rn(__ddiv_rn(sum, static_cast<double>(a.N)));
-                vmax[c] = mx;
+                const float m = __double2float_rn(__ddiv_rn(sum, static_cast<double>(a.N)));
+                mu[c] = m;
                 vinv[c] = mx > 0.f ? 448.f / mx : 0.f;
-            }
-            cur_bh = bh;
-        }
-        if (threadIdx.x == 0 && !bad) {
-            if (wait_one(&bar[buf], (k >> 1) & 1, a.err, &abort_st, false, 0))
-                waited = k + 1;
-            else
-                bad = 1;
-        }
-        // the rows and the statistics are ready, and every thread is done with
-        // the previous item, so its buffer takes the next item's rows
-        __syncthreads();
-        if (threadIdx.x == 0 && !bad && item + 1 < i1) {
-            issue(item + 1, buf ^ 1);
-            ++issued;
-        }
-        if (blk == 0 && (DO_K || DO_V)) {
-            for (int c = threadIdx.x; c < D; c += NTH) {
-                if (DO_K) {
-                    a.ws_k_mean[bh * D + c] = mu[c];
-                    if (a.user_k_mean) a.user_k_mean[bh * D + c] = mu[c];
-                }
-                if (DO_V) {
-                    a.ws_v_inv[bh * D + c] = vinv[c];
-                    a.c.v_scale[bh * D + c] = vmax[c] > 0.f ? vmax[c] / 448.f : 0.f;
+                if (c0 == 0) {  // one CTA writes the per-head outputs
+                    if (DO_K && a.user_k_mean) a.user_k_mean[(int64_t)h * D + c] = m;
+                    if (DO_V) a.c.v_scale[(int64_t)h * D + c] = mx > 0.f ? mx / 448.f : 0.f;
                 }
             }
+            __syncthreads();
         }
-        const int row0 = blk * kQBlock;
-        const uint16_t *base = bufs + buf * NT * TILE;
-
-        // Q and the smoothed K of this thread's rows stay in registers from the
-        // maximum to the codes; one block reduction serves Q and both K blocks.
-        float qv[DO_Q ? NI : 1][8], kv[DO_K ? NI : 1][8];
-        float qa = 0.f, ka0 = 0.f, ka1 = 0.f;
-        if (!bad) {
-            if (DO_Q) {
+        const int b = h / a.H, hh = h % a.H;
+        for (int u = c1 - 1 - grp; u >= c0; u -= Gm::GROUPS) {
+            const int rbase = u * kQBlock + gw * RB + rl;  // this lane's first row
+            const int64_t obase = ((int64_t)h * a.n_pad + rbase) * D + vec * 8;
+            // all of the block's rows are requested at once: one memory latency per block
+            uint4 xq[DO_Q ? NB : 1], xk[DO_K ? NB : 1], xv[DO_V ? NB : 1];
+            if constexpr (DO_Q) load_rows<NB, RPI>(xq, a.q.p + b * a.q.sb + hh * a.q.sh + vec * 8, a.q.sn, rbase, a.N, drop);
+            if constexpr (DO_K) load_rows<NB, RPI>(xk, a.k.p + b * a.k.sb + hh * a.k.sh + vec * 8, a.k.sn, rbase, a.N, drop);
+            if constexpr (DO_V) load_rows<NB, RPI>(xv, a.v.p + b * a.v.sb + hh * a.v.sh + vec * 8, a.v.sn, rbase, a.N, drop);
+            if constexpr (DO_Q) {
+                const uint4 *x = xq;
+                uint32_t am = 0u;
 #pragma unroll
-                for (int i = 0; i < NI; ++i) {
-                    unpack8(ld_tile(base + OQ * TILE, tile_off(kQBlock, r0 + i * RPI, cv)), qv[i]);
+                for (int i = 0; i < NB; ++i)
+                    am = bmax_abs(bmax_abs(bmax_abs(bmax_abs(am, x[i].x), x[i].y), x[i].z), x[i].w);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) qa = fmaxf(qa, fabsf(qv[i][e]));
+                for (int o = 16; o > 0; o >>= 1) am = bmax_abs(am, __shfl_xor_sync(0xffffffffu, am, o));
+                float qa = fmaxf(bf_bits(am & 0xffffu), bf_bits(am >> 16));
+                // the block's maximum over the group's warps
+                if (lane == 0) grp_max[grp][parity][0][gw] = qa;
+                group_sync(1 + grp, 32 * WU);
+#pragma unroll
+                for (int w = 0; w < WU; ++w) qa = fmaxf(qa, grp_max[grp][parity][0][w]);
+                const float inv = qa > 0.f ? 127.f / qa : 0.f;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    float f[8];
+                    unpack8(x[i], f);
+                    *reinterpret_cast<uint2 *>(a.c.q_i8 + obase + (int64_t)i * RPI * D) = i8x8(f, inv);
                 }
+                if (gw == 0 && lane == 0) a.c.q_scale[(int64_t)h * nqb + u] = qa > 0.f ? qa / 127.f : 0.f;
             }
-            if (DO_K) {
-                float m8[8];
+            if constexpr (DO_K) {
+                // the warp's rows lie in one 64-token K block, shared by KW warps
+                const uint4 *x = xk;
+                float mu8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) m8[e] = mu[cv * 8 + e];
+                for (int e = 0; e < 8; ++e) mu8[e] = mu[vec * 8 + e];
+                float ka = 0.f;
 #pragma unroll
-                for (int i = 0; i < NI; ++i) {
-                    const int row = r0 + i * RPI;
-                    if (row0 + row < a.N) {  // rows past N stay zero (not -mean)
+                for (int i = 0; i < NB; ++i) {
+                    if (rbase + i * RPI < a.N) {  // rows past N stay zero (not -mean)
+                        float f[8], d[8];
+                        unpack8(x[i], f);
+#pragma unroll
+                        for (int e = 0; e < 8; e += 2) fsub2(d[e], d[e + 1], f[e], f[e + 1], mu8[e], mu8[e + 1]);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) ka = fmaxf(ka, fabsf(d[e]));
+                    }
+                }
+                ka = warp_fmax(ka);
+                if (KW > 1) {
+                    if (lane == 0) grp_max[grp][parity][1][gw] = ka;
+                    group_sync(1 + grp, 32 * WU);
+                    const int w0 = gw - gw % KW;
+#pragma unroll
+                    for (int w = 0; w < KW; ++w) ka = fmaxf(ka, grp_max[grp][parity][1][w0 + w]);
+                }
+                const float inv = ka > 0.f ? 127.f / ka : 0.f;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    float d[8];
+                    if (rbase + i * RPI < a.N) {
                         float f[8];
-                        unpack8(ld_tile(base + OK * TILE, tile_off(kQBlock, row, cv)), f);
+                        unpack8(x[i], f);
 #pragma unroll
-                        for (int e = 0; e < 8; e += 2) fsub2(kv[i][e], kv[i][e + 1], f[e], f[e + 1], m8[e], m8[e + 1]);
+                        for (int e = 0; e < 8; e += 2) fsub2(d[e], d[e + 1], f[e], f[e + 1], mu8[e], mu8[e + 1]);
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) kv[i][e] = 0.f;
+                        for (int e = 0; e < 8; ++e) d[e] = 0.f;
                     }
-                    float am = 0.f;
+                    *reinterpret_cast<uint2 *>(a.c.k_i8 + obase + (int64_t)i * RPI * D) = i8x8(d, inv);
+                }
+                if (gw % KW == 0 && lane == 0)
+                    a.c.k_scale[(int64_t)h * nkb + (u * kQBlock + gw * RB) / kKBlock] = ka > 0.f ? ka / 127.f : 0.f;
+            }
+            if constexpr (DO_V) {
+                const uint4 *x = xv;
+                float vi8[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(kv[i][e]));
-                    if (row < kKBlock) ka0 = fmaxf(ka0, am); else ka1 = fmaxf(ka1, am);
+                for (int e = 0; e < 8; ++e) vi8[e] = vinv[vec * 8 + e];
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    float f[8];
+                    unpack8(x[i], f);
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        // IEEE products (nothing is added); the conversion is
+                        // volatile so that the vectors are coded one after
+                        // another, not all unpacked at once
+                        const float y0 = __fmul_rn(f[e], vi8[e]), y1 = __fmul_rn(f[e + 1], vi8[e + 1]);
+                        w[e / 2] = e4m3x2(y0, y1);
+                    }
+                    *reinterpret_cast<uint2 *>(a.c.v_e4m3 + obase + (int64_t)i * RPI * D) =
+                        make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
                 }
             }
-            block_max3_n<NTH>(qa, ka0, ka1, red, k & 1);
-        }
-
-        if (DO_Q && !bad) {
-            const float inv = qa > 0.f ? 127.f / qa : 0.f;
-            int8_t *dst = a.c.q_i8 + ((int64_t)bh * a.n_pad + row0) * D + cv * 8;
-#pragma unroll
-            for (int i = 0; i < NI; ++i)
-                *reinterpret_cast<uint2 *>(dst + (int64_t)(r0 + i * RPI) * D) = i8x8(qv[i], inv);
-            if (threadIdx.x == 0) a.c.q_scale[(int64_t)bh * nqb + blk] = qa > 0.f ? qa / 127.f : 0.f;
-        }
-
-        if (DO_K && !bad) {
-            const float inv0 = ka0 > 0.f ? 127.f / ka0 : 0.f;
-            const float inv1 = ka1 > 0.f ? 127.f / ka1 : 0.f;
-            int8_t *dst = a.c.k_i8 + ((int64_t)bh * a.n_pad + row0) * D + cv * 8;
-#pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                const int row = r0 + i * RPI;
-                *reinterpret_cast<uint2 *>(dst + (int64_t)row * D) = i8x8(kv[i], row < kKBlock ? inv0 : inv1);
-            }
-            if (threadIdx.x == 0) {
-                a.c.k_scale[(int64_t)bh * nkb + 2 * blk] = ka0 > 0.f ? ka0 / 127.f : 0.f;
-                a.c.k_scale[(int64_t)bh * nkb + 2 * blk + 1] = ka1 > 0.f ? ka1 / 127.f : 0.f;
-            }
-        }
-
-        if (DO_V && !bad) {
-            const uint16_t *tile = base + OV * TILE;
-            float inv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) inv[e] = vinv[cv * 8 + e];
-            uint8_t *dst = a.c.v_e4m3 + ((int64_t)bh * a.n_pad + row0) * D + cv * 8;
-#pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                float f[8];
-                unpack8(ld_tile(tile, tile_off(kQBlock, r0 + i * RPI, cv)), f);
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 8; e += 2) {
-                    float y0, y1;
-                    fmul2(y0, y1, f[e], f[e + 1], inv[e], inv[e + 1]);  // IEEE products; nothing is added
-                    uint16_t pr;
-                    // cvt packs its first source in the high byte: (hi=e+1, lo=e)
-                    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(pr) : "f"(y1), "f"(y0));
-                    w[e / 2] = pr;
-                }
-                *reinterpret_cast<uint2 *>(dst + (int64_t)(r0 + i * RPI) * D) =
-                    make_uint2(w[0] | (w[1] << 16), w[2] | (w[3] << 16));
-            }
+            parity ^= 1;
         }
     }
-    if (threadIdx.x == 0) {
-        // every copy started here lands before the CTA exits
-        for (int k = waited; k < issued; ++k) wait_one(&bar[k & 1], (k >> 1) & 1, a.err, &abort_st, true, 0);
-    }
-}
-
-// Raise a kernel's dynamic shared-memory limit on the current device once:
-// the attribute belongs to the device, so `done` keeps one bit per device
-// index (indices past 63 set it on every call).
-template <typename K>
-cudaError_t ensure_smem_limit(K kern, int smem, std::atomic<uint64_t> &done) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    const uint64_t bit = dev >= 0 && dev < 64 ? (1ull << dev) : 0ull;
-    if (bit && (done.load(std::memory_order_relaxed) & bit)) return cudaSuccess;
-    if ((e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) != cudaSuccess) return e;
-    done.fetch_or(bit, std::memory_order_relaxed);
-    return cudaSuccess;
-}
-
-// CTAs that fit at once on the device for a kernel and its dynamic shared memory.
-template <typename K>
-int resident_ctas(K kern, int threads, int smem) {
-    int dev = 0, sms = 0, per_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, smem) != cudaSuccess)
-        return 0;
-    return sms * per_sm;
-}
-
-template <int D>
-cudaError_t launch_stats_d(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, cudaStream_t st) {
-    CUtensorMap tk, tv;
-    StatsArgs a{};
-    cudaError_t e;
-    if (k && (e = make_bf16_token_map(&tk, *k, s, kRowsPerLoad, &a.k_swap)) != cudaSuccess) return e;
-    if (v && (e = make_bf16_token_map(&tv, *v, s, kRowsPerLoad, &a.v_swap)) != cudaSuccess) return e;
-    if (!k) tk = tv;
-    if (!v) tv = tk;
-    a.H = s.H;
-    a.BH = s.BH();
-    a.N = s.N;
-    a.nch = s.n_chunks();
-    a.chunk = s.chunk_rows();
-    a.do_k = k != nullptr;
-    a.do_v = v != nullptr;
-    a.ksum_part = ws.ksum_part;
-    a.vmax_part = ws.vmax_part;
-    if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
-    constexpr int RPI = kThreads / (D / 8);
-    const int smem = kStatsStages * 2 * kRowsPerLoad * D * 2 + (kThreads / 32) * D * 8 + RPI * D * 4;
-    static std::atomic<uint64_t> limit_set{0};  // one per instantiation
-    if ((e = ensure_smem_limit(k_stats<D>, smem, limit_set)) != cudaSuccess) return e;
-    const int items = a.nch * s.BH();
-    const int ctas = resident_ctas(k_stats<D>, kThreads, smem);
-    if (ctas <= 0) return cudaErrorInvalidConfiguration;
-    a.per = (items + ctas - 1) / ctas;
-    k_stats<D><<<(items + a.per - 1) / a.per, kThreads, smem, st>>>(tk, tv, a);
-    return cudaGetLastError();
 }
 
 template <int D, bool DQ, bool DK, bool DV>
-cudaError_t launch_quant_k(const Shape &s, const CUtensorMap &tq, const CUtensorMap &tk, const CUtensorMap &tv,
-                           QuantArgs a, cudaStream_t st) {
-    constexpr int NT = (DQ ? 1 : 0) + (DK ? 1 : 0) + (DV ? 1 : 0);
-    const int smem = 2 * NT * kQBlock * D * 2;
-    auto kern = k_quant<D, DQ, DK, DV>;
-    static std::atomic<uint64_t> limit_set{0};  // one per instantiation
+cudaError_t launch_qpass_k(const Shape &s, const PassArgs &a, cudaStream_t st) {
+    auto kern = k_qpass<D, DQ, DK, DV>;
+    int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e;
-    if ((e = ensure_smem_limit(kern, smem, limit_set)) != cudaSuccess) return e;
-    const int items = s.n_qblocks() * s.BH();
-    const int ctas = resident_ctas(kern, quant_threads<D>(), smem);
-    if (ctas <= 0) return cudaErrorInvalidConfiguration;
-    a.per = (items + ctas - 1) / ctas;
-    return launch_dependent(kern, dim3((items + a.per - 1) / a.per), dim3(quant_threads<D>()), smem, st, tq, tk, tv,
-                            a);
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kPassThreads, 0)) != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    // every CTA is resident at once (cooperative launch), so a CTA waiting on
+    // another's phase-A partials never waits on one that has not started; no
+    // more CTAs than 128-token blocks, nor than the statistics slots allow
+    const long long grid = std::min<long long>(
+        {(long long)sms * per_sm, (long long)s.BH() * s.n_qblocks(), (long long)kStatsMaxGrid});
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kPassThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeCooperative;
+    at[0].val.cooperative = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+// A 48-bit stamp per call from a process-wide counter that starts at a
+// clock-derived value; bit 47 is always set, so a zeroed flag never matches.
+unsigned long long next_stamp() {
+    static std::atomic<unsigned long long> counter{
+        static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count())};
+    const unsigned long long v = counter.fetch_add(1, std::memory_order_relaxed) + 1;
+    return (v & ((1ull << 48) - 1)) | (1ull << 47);
 }
 
 template <int D>
-cudaError_t launch_quant_d(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
+cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
                            float *user_k_mean, const Codes &c, cudaStream_t st) {
-    CUtensorMap tq, tk, tv;
-    QuantArgs a{};
-    cudaError_t e;
-    if (q && (e = make_bf16_token_map(&tq, *q, s, kRowsPerLoad, &a.q_swap)) != cudaSuccess) return e;
-    if (k && (e = make_bf16_token_map(&tk, *k, s, kRowsPerLoad, &a.k_swap)) != cudaSuccess) return e;
-    if (v && (e = make_bf16_token_map(&tv, *v, s, kRowsPerLoad, &a.v_swap)) != cudaSuccess) return e;
-    const CUtensorMap &any = q ? tq : (k ? tk : tv);
-    if (!q) tq = any;
-    if (!k) tk = any;
-    if (!v) tv = any;
+    PassArgs a{};
+    const Src none{nullptr, 0, 0, 0};
+    a.q = q ? *q : none;
+    a.k = k ? *k : none;
+    a.v = v ? *v : none;
     a.H = s.H;
     a.BH = s.BH();
     a.N = s.N;
     a.n_pad = s.n_pad();
-    a.nch = s.n_chunks();
     a.ksum_part = ws.ksum_part;
     a.vmax_part = ws.vmax_part;
-    a.ws_k_mean = ws.k_mean;
-    a.ws_v_inv = ws.v_inv;
+    a.flags = ws.flags;
+    a.stamp = next_stamp();
     a.user_k_mean = user_k_mean;
     a.c = c;
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
-    if (q && k && v) return launch_quant_k<D, true, true, true>(s, tq, tk, tv, a, st);
-    if (q && k && !v) return launch_quant_k<D, true, true, false>(s, tq, tk, tv, a, st);
-    if (!q && k && v) return launch_quant_k<D, false, true, true>(s, tq, tk, tv, a, st);
-    if (!q && !k && v) return launch_quant_k<D, false, false, true>(s, tq, tk, tv, a, st);
-    if (q && !k && v) return launch_quant_k<D, true, false, true>(s, tq, tk, tv, a, st);
+    if (q && k && v) return launch_qpass_k<D, true, true, true>(s, a, st);
+    if (q && k && !v) return launch_qpass_k<D, true, true, false>(s, a, st);
+    if (!q && k && v) return launch_qpass_k<D, false, true, true>(s, a, st);
+    if (!q && !k && v) return launch_qpass_k<D, false, false, true>(s, a, st);
+    if (q && !k && v) return launch_qpass_k<D, true, false, true>(s, a, st);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-cudaError_t launch_stats(const Shape &s, const Src *k, const Src *v, const StatsWs &ws, cudaStream_t st) {
-    return s.d == 128 ? launch_stats_d<128>(s, k, v, ws, st) : launch_stats_d<64>(s, k, v, ws, st);
-}
-
-cudaError_t launch_quant(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
+cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
                          float *user_k_mean, const Codes &c, cudaStream_t st) {
-    return s.d == 128 ? launch_quant_d<128>(s, q, k, v, ws, user_k_mean, c, st)
-                      : launch_quant_d<64>(s, q, k, v, ws, user_k_mean, c, st);
+    return s.d == 128 ? launch_qpass_d<128>(s, q, k, v, ws, user_k_mean, c, st)
+                      : launch_qpass_d<64>(s, q, k, v, ws, user_k_mean, c, st);
 }
 
 }  // namespace sage

@@ -27,7 +27,7 @@ def L():
 def test_noalloc_rejects_a_shape_beyond_its_scratch(L):
     st = (ctypes.c_int64 * 4)(128 * 128 * 128, 128 * 128, 128, 1)
     p = ctypes.c_void_p(16 * 4096)
-    # with B*H = 4096 heads the per-head statistics alone need 8 MB, twice the array
+    # with B*H = 4096 heads the statistics slots need about 7 MB, more than the array
     assert sage.sage_quant_workspace_bytes(32, 128, 128, 128) > 4 << 20
     rc = L.sage_quant_qk_noalloc(p, st, p, st, 32, 128, 128, 128, p, p, p, p, None, None)
     assert rc == 3
@@ -35,22 +35,31 @@ def test_noalloc_rejects_a_shape_beyond_its_scratch(L):
 
 
 def test_noalloc_scratch_bound_on_the_workloads(L):
-    """The scratch a shape needs is the documented formula; the video and 64K
-    workloads need more than the 4 MiB array and are rejected with status 3
-    (before any launch), the smaller ones fit."""
+    """The scratch a shape needs is the documented formula; every workload
+    fits the 4 MiB array, and the largest head count that fits is the one the
+    header states (about 2200 heads at d = 128, 4900 at d = 64): one more head
+    is rejected with status 3 before any launch."""
     up = lambda x: -(-x // 1024) * 1024
+
+    def need(B, H, N, d):
+        S = B * H + min(512, B * H * -(-N // 128))
+        return up(8 * S * d) + up(4 * S * d) + up(8 * S)
+
     for name, w in WORKLOADS.items():
-        C = -(-w.N // 256)
-        need = up(8 * w.B * w.H * C * w.d) + up(4 * w.B * w.H * C * w.d) + 2 * up(4 * w.B * w.H * w.d)
-        assert sage.sage_quant_workspace_bytes(w.B, w.H, w.N, w.d) == need, name
-        assert (need <= 4 << 20) == (name not in ("video", "long64k")), name
-    w = WORKLOADS["video"]
-    st = (ctypes.c_int64 * 4)(w.N * 3 * w.H * w.d, w.d, 3 * w.H * w.d, 1)
-    p = ctypes.c_void_p(16 * 4096)
-    rc = L.sage_quant_qk_noalloc(p, st, p, st, w.B, w.H, w.N, w.d, p, p, p, p, None, None)
-    assert rc == 3
-    assert b"scratch" in L.sage_last_error_message()
+        assert sage.sage_quant_workspace_bytes(w.B, w.H, w.N, w.d) == need(w.B, w.H, w.N, w.d), name
+        assert need(w.B, w.H, w.N, w.d) <= 4 << 20, name
+    for d, near in ((128, 2200), (64, 4900)):
+        fit = max(h for h in range(near - 50, near + 50) if need(1, h, 4096, d) <= 4 << 20)
+        assert abs(fit - near) <= 10, (d, fit)
+        assert sage.sage_quant_workspace_bytes(1, fit + 1, 4096, d) > 4 << 20
+        st = (ctypes.c_int64 * 4)((fit + 1) * 4096 * d, 4096 * d, d, 1)
+        p = ctypes.c_void_p(16 * 4096)
+        rc = L.sage_quant_qk_noalloc(p, st, p, st, 1, fit + 1, 4096, d, p, p, p, p, None, None)
+        assert rc == 3, (d, rc)
+        assert b"scratch" in L.sage_last_error_message()
     # a shape the library does not take at all is reported as such, not as scratch
+    st = (ctypes.c_int64 * 4)(128 * 70000 * 128, 128 * 128, 128, 1)
+    p = ctypes.c_void_p(16 * 4096)
     assert L.sage_quant_qk_noalloc(p, st, p, st, 1, 70000, 128, 128, p, p, p, p, None, None) == 2
 
 
