@@ -40,7 +40,7 @@ DTYPE = "i8/e4m3"        # QK^T on int8 codes, PV on e4m3 codes; bf16 in and out
 PRIMARY = "flux"
 SECONDARIES = ("video", "long16k", "long64k")
 PEAK_NOTE = "measured cuBLAS bf16 burst x 2 (nominal 8-bit/bf16 dense ratio)"
-LAUNCHES_PER_STEP = 3    # k_stats (partial K/V statistics), k_quant (finishes them, codes), k_attn
+LAUNCHES_PER_STEP = 2    # k_qpass (K/V statistics, then the codes), k_attn
 
 
 def _env_int(name, default):

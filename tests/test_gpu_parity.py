@@ -325,6 +325,75 @@ def test_back_to_back_forwards_sharing_a_workspace_do_not_interfere():
         assert torch.equal(a.view(torch.int16), o.view(torch.int16))
 
 
+@pytest.mark.parametrize("B,H,N,d,layout", [(1, 24, 4608, 128, "fused"), (1, 2, 16384, 128, "contiguous"),
+                                             (2, 5, 1000, 64, "contiguous")])
+def test_quantize_pass_ignores_what_the_workspace_held(B, H, N, d, layout):
+    """The quantize kernel's CTAs publish their statistics through flags in the
+    workspace, stamped per call; whatever the workspace held before (zeros,
+    all ones, random bytes, or the leftovers of another shape's call) must not
+    change a bit of the result.  (1, 2, 16384) puts ~74 CTAs on each head, so
+    every flag has many readers."""
+    w = tiny_custom(B, H, N, d, seed=811, layout=layout, bias_sigma=2.0, outlier_frac=0.02)
+    _, (qd, kd, vd), _ = _inputs(w)
+    ref = sage.sage_attn_fwd(qd, kd, vd)
+    ref_q = sage.sage_quant_qk(qd, kd)
+    torch.cuda.synchronize()
+    nbytes = sage.sage_attn_workspace_bytes(B, H, N, d)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=DEV)
+    g = torch.Generator(device=DEV).manual_seed(5)
+    other = tiny_custom(1, 3, 700, d, seed=812)
+    _, (qo, ko, vo), _ = _inputs(other)
+    fills = [lambda: ws.fill_(0), lambda: ws.fill_(255),
+             lambda: ws.copy_(torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device=DEV, generator=g)),
+             lambda: sage.sage_attn_fwd(qo, ko, vo, workspace=ws)]
+    for fill in fills:
+        fill()
+        out = sage.sage_attn_fwd(qd, kd, vd, workspace=ws)
+        qws = torch.empty(sage.sage_quant_workspace_bytes(B, H, N, d), dtype=torch.uint8, device=DEV)
+        qws.fill_(255)
+        got_q = sage.sage_quant_qk(qd, kd, workspace=qws)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+        for key in ("q_i8", "q_scale", "k_i8", "k_scale", "k_mean"):
+            assert torch.equal(got_q[key], ref_q[key]), key
+
+
+def test_forward_replays_from_a_cuda_graph():
+    """A captured forward replays the same kernel arguments, so the quantize
+    kernel's per-call stamp repeats; its flags are cleared by their last
+    reader within each launch, so every replay waits for its own statistics.
+    Three inputs are copied into the captured buffers in turn; each replay
+    must equal the eager forward of the same input bit for bit."""
+    ws_ = [tiny_custom(1, 24, 4608, 128, seed=90 + i, layout="contiguous", bias_sigma=2.0) for i in range(3)]
+    ins = [_inputs(w)[1] for w in ws_]
+    eager = []
+    for (qd, kd, vd) in ins:
+        eager.append(sage.sage_attn_fwd(qd, kd, vd))
+    q, k, v = (t.clone() for t in ins[0])
+    out = torch.empty_like(eager[0])
+    ws = torch.empty(sage.sage_attn_workspace_bytes(1, 24, 4608, 128), dtype=torch.uint8, device=DEV)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up on the capture stream (first-call set-up outside the capture)
+        sage.sage_attn_fwd(q, k, v, out=out, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        sage.sage_attn_fwd(q, k, v, out=out, workspace=ws)
+    for rep in range(2):
+        for (qd, kd, vd), want in zip(ins, eager):
+            q.copy_(qd)
+            k.copy_(kd)
+            v.copy_(vd)
+            graph.replay()
+            torch.cuda.synchronize()
+            sage.sage_check()
+            assert torch.equal(out.view(torch.int16), want.view(torch.int16)), rep
+    del graph
+
+
 # --------------------------------------------------------------------------- dense reference and exact
 
 @pytest.mark.parametrize("name", ["tiny", "sdxl"])
