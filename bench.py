@@ -78,6 +78,70 @@ def _attn_traffic(workload):
     return int(w["dram_bytes_read"]) + int(w["dram_bytes_write"])
 
 
+EX2_PER_SCORE = 0.75     # the softmax takes 2^x on the MUFU unit for 6 of every 8 scores, by polynomial for 2
+
+
+def _attn_instructions(d):
+    """Warp instructions per score of the dense attention kernel at head dim d,
+    as counted by ncu (profiles/k_attn_instructions.txt), or None when there is
+    no count or the kernel source changed since it was taken."""
+    import hashlib
+    here = os.path.dirname(os.path.abspath(__file__))
+    try:
+        with open(os.path.join(here, "profiles", "k_attn_instructions.txt")) as f:
+            rec = json.load(f)
+        with open(os.path.join(here, "quantized_attention_qk_b200", "csrc", "sage_attn.cu"), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, ValueError):
+        return None
+    e = rec.get("head_dims", {}).get(str(d))
+    if rec.get("source_sha256") != sha or not e:
+        return None
+    return float(e["warp_instructions"]) / float(e["scores"])
+
+
+def _ex2_rate(dev):
+    """Exponentials per second of the exponential unit, measured here: the
+    library's ex2 probe (the softmax's own ex2.approx.ftz instruction, eight
+    independent chains per thread, 8 CTAs of 256 threads per SM), 2 untimed
+    and 5 timed launches, CUDA events on the current stream."""
+    import torch
+
+    import quantized_attention_qk_b200 as sage
+
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    blocks, iters = 8 * sms, 2048
+    sink = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+    for _ in range(2):
+        sage.sage_debug_ex2_probe(sink, blocks, iters)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(5):
+        sage.sage_debug_ex2_probe(sink, blocks, iters)
+    e1.record()
+    torch.cuda.synchronize()
+    return 5 * blocks * 256 * iters * 8 / (e0.elapsed_time(e1) * 1e-3)
+
+
+def _softmax_roofline(w, attn_ms, kept, ex2_rate, sm_mhz, sms, instr_per_score):
+    """The attention kernel against its softmax ceilings, in scores per second:
+    the exponential unit (measured rate / EX2_PER_SCORE) and the issue slots
+    (four warp instructions per SM and clock at the sampled SM clock, over the
+    kernel's own warp instructions per score; none when there is no count for
+    this source and head dim)."""
+    achieved = kept * w.B * w.H * w.N * w.N / (attn_ms * 1e-3)
+    ceilings = {"ex2": ex2_rate / EX2_PER_SCORE}
+    if instr_per_score and sm_mhz:
+        ceilings["issue"] = 4.0 * sms * sm_mhz * 1e6 / instr_per_score
+    peak = min(ceilings.values())
+    return {"bound": "alu", "unit": "Tscores/s", "achieved": round(achieved / 1e12, 4),
+            "peak": round(peak / 1e12, 4), "frac": round(achieved / peak, 4),
+            "ceilings": {k: round(v / 1e12, 4) for k, v in ceilings.items()},
+            "ex2_measured_per_s": round(ex2_rate / 1e12, 4), "ex2_per_score": EX2_PER_SCORE,
+            "warp_instructions_per_score": None if instr_per_score is None else round(instr_per_score, 5),
+            "sm_mhz": sm_mhz}
+
+
 def _workload_desc(w):
     return f"{w.name}: B={w.B} H={w.H} N={w.N} d={w.d} {w.layout} qkv"
 
@@ -339,6 +403,15 @@ def run_gpu(args):
 
     wp = WORKLOADS[args.workload]
     r = measure(wp, args.steps, args.warmup)
+    # the softmax's ceilings (outside every timed region): the exponential
+    # unit measured here, the issue slots from the kernel's counted instructions
+    ex2_rate = _ex2_rate(dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    dense = args.tau is None and not args.kres and not args.fused_q
+
+    def softmax_roofline(w, rr):
+        return _softmax_roofline(w, rr["attn_ms"], rr["kept"], ex2_rate, rr["clocks"].get("sm_mhz"), sms,
+                                 _attn_instructions(w.d) if dense else None)
     ms = r["total_ms"] / args.steps
     value = whole_job_tops(world, wp.ops, args.steps, r["total_ms"])
     attn_tops = r["kept"] * wp.ops / (r["attn_ms"] * 1e-3) / 1e12  # the kernel's own work
@@ -354,6 +427,7 @@ def run_gpu(args):
                      "traffic": None if (args.tau is not None or args.kres or args.fused_q) else _attn_traffic(wp.name),
                      "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
+        "roofline_softmax": softmax_roofline(wp, r),
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
@@ -386,6 +460,7 @@ def run_gpu(args):
                 "unit": "TOPS", "ms_per_step": round(r2["total_ms"] / k2, 4), "steps": k2,
                 "attn_tops": round(attn_tops2, 2), "attn_ms": round(r2["attn_ms"], 4),
                 "attn_frac": round(attn_tops2 / peak_8bit, 4),
+                "softmax_frac": softmax_roofline(ws_, r2)["frac"],
                 "e2e_tops": round(world * ws_.ops / (r2["e2e_ms"] * 1e-3) / 1e12, 2), "clocks": r2["clocks"]})
             line["gpu_launches"] += LAUNCHES_PER_STEP * k2
     if rank == 0 and world == 1 and args.cpu_baseline:

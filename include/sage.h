@@ -427,6 +427,19 @@ sage_status_t sage_debug_qk_tile(const int8_t *q_i8, const int8_t *k_i8,
  */
 sage_status_t sage_debug_wait_timeout(int microseconds, sage_stream_t stream);
 
+/*
+ * sage_debug_ex2_probe -- a throughput probe of the exponential unit, for
+ * stating the softmax's ceiling next to the attention kernel's time: `blocks`
+ * CTAs of 256 threads, each thread running eight independent chains of
+ * `iters` base-2 exponentials (the ex2.approx.ftz instruction the softmax
+ * issues), i.e. blocks * 256 * iters * 8 exponentials; the caller times the
+ * launch on `stream`.  sink: device float[blocks * 256] on the current device
+ * (4-byte aligned), written with the chains' sums.  blocks 1..65535, iters
+ * 1..2^20 (SAGE_ERR_INVALID_ARG otherwise).  Asynchronous; not part of any
+ * forward.
+ */
+sage_status_t sage_debug_ex2_probe(float *sink, int blocks, int iters, sage_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

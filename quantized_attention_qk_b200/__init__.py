@@ -71,6 +71,7 @@ _SIGS = {
     "sage_tau_schedule": ([_I32, _I32, ctypes.c_float, ctypes.c_float], ctypes.c_float),
     "sage_attn_kres_workspace_bytes": ([_I32] * 4, _SZ),
     "sage_debug_wait_timeout": ([_I32, _P], _I32),
+    "sage_debug_ex2_probe": ([_P, _I32, _I32, _P], _I32),
     "sage_attn_fwd_fused_q": ([_P, _I64P, _P, _I64P, _P, _I64P, _P, _I64P, _I32, _I32, _I32, _I32, ctypes.c_float,
                                _P, _SZ, _P, _P, _P], _I32),
     "sage_quant_k_residual": ([_P, _I64P, _I32, _I32, _I32, _I32, _P, _P, _P, _P], _I32),
@@ -454,3 +455,14 @@ def sage_debug_wait_timeout(microseconds: int = 10000, stream=None, device=None)
     the stream reports SAGE_ERR_TIMEOUT."""
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     _run(dev, lib().sage_debug_wait_timeout, int(microseconds), _stream(stream, dev))
+
+
+def sage_debug_ex2_probe(sink, blocks: int, iters: int, stream=None):
+    """Launch the exponential-unit throughput probe: ``blocks`` CTAs of 256
+    threads, each running eight chains of ``iters`` base-2 exponentials
+    (blocks * 256 * iters * 8 in all) into ``sink`` (float32 device tensor of
+    at least blocks * 256 elements).  The caller times it."""
+    if sink.dtype != torch.float32 or not sink.is_cuda or sink.numel() < blocks * 256:
+        raise ValueError("sink must be a float32 CUDA tensor of at least blocks * 256 elements")
+    dev = sink.device
+    _run(dev, lib().sage_debug_ex2_probe, _ptr(sink), int(blocks), int(iters), _stream(stream, dev))

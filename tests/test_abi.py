@@ -159,10 +159,15 @@ def test_mask_packing_round_trips():
         assert bool(((m[0, 0, 0, j // 32].item() & 0xFFFFFFFF) >> (j % 32)) & 1) == bool(keep[0, 0, 0, j])
 
 
-def test_wait_probe_rejects_out_of_range_limits_before_any_launch(L):
+def test_probes_reject_out_of_range_arguments_before_any_launch(L):
     for us in (0, -5, 1000001):
         assert L.sage_debug_wait_timeout(us, None) == 1
         assert "microseconds" in L.sage_last_error_message().decode()
+    p = ctypes.c_void_p(16 * 4096)
+    for blocks, iters in ((0, 10), (70000, 10), (1, 0), (1, (1 << 20) + 1)):
+        assert L.sage_debug_ex2_probe(p, blocks, iters, None) == 1
+    assert L.sage_debug_ex2_probe(None, 1, 1, None) == 1
+    assert L.sage_debug_ex2_probe(ctypes.c_void_p(16 * 4096 + 2), 1, 1, None) == 1
 
 
 def test_missing_library_fails_loudly(tmp_path, monkeypatch):

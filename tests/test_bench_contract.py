@@ -28,3 +28,29 @@ def test_reference_arm_prints_one_contract_line():
     e = d["e2e"]
     assert e["value"] == d["value"] and e["unit"] == d["unit"]
     assert e["h2d_bytes_per_step"] == 0 and e["d2h_bytes_per_step"] == 0
+
+
+def test_softmax_roofline_takes_the_lower_ceiling():
+    """The attention kernel against its softmax ceilings: the exponential unit
+    (measured rate / exponentials per score) and the issue slots (four warp
+    instructions per SM and clock over the kernel's warp instructions per
+    score); achieved scores per second over the lower one."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_attention_qk_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["flux"]
+    scores = w.B * w.H * w.N * w.N
+    r = bench._softmax_roofline(w, attn_ms=0.2, kept=1.0, ex2_rate=4.0e12, sm_mhz=2000.0, sms=148,
+                                instr_per_score=0.25)
+    assert abs(r["achieved"] - scores / 0.2e-3 / 1e12) < 1e-4
+    assert abs(r["ceilings"]["ex2"] - 4.0 / bench.EX2_PER_SCORE) < 1e-4
+    assert abs(r["ceilings"]["issue"] - 4 * 148 * 2.0e9 / 0.25 / 1e12) < 1e-4
+    assert r["peak"] == min(r["ceilings"].values())
+    assert abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-3
+    # without an instruction count only the exponential ceiling is stated
+    r2 = bench._softmax_roofline(w, 0.2, 1.0, 4.0e12, 2000.0, 148, None)
+    assert set(r2["ceilings"]) == {"ex2"} and r2["peak"] == r2["ceilings"]["ex2"]
+    # a kept fraction (block-sparse) scales the scores the kernel computed
+    r3 = bench._softmax_roofline(w, 0.2, 0.5, 4.0e12, 2000.0, 148, None)
+    assert abs(r3["achieved"] - r2["achieved"] / 2) < 1e-4
