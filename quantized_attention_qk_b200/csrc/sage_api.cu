@@ -469,7 +469,14 @@ sage_status_t sage_quant_k_residual(const void *k_bf16, const int64_t k_stride[4
         (r = check_on_current_device(k_i8, "k_i8")))
         return r;
     const Shape s{B, H, N, d};
-    cudaError_t e = launch_kres(s, src(k_bf16, k_stride), k_i8, k_scale, k_bmean, reinterpret_cast<cudaStream_t>(stream));
+    // K alone needs no statistics (each block's mean is its own), so no scratch
+    const Src ks = src(k_bf16, k_stride);
+    const StatsWs none{};
+    Codes c{};
+    c.k_i8 = k_i8;
+    c.k_scale = k_scale;
+    cudaError_t e = launch_qpass(s, nullptr, &ks, nullptr, none, nullptr, c, reinterpret_cast<cudaStream_t>(stream),
+                                 k_bmean);
     if (e != cudaSuccess) return cuda_fail(e, "K-residual quantization");
     return SAGE_OK;
 }
@@ -497,10 +504,8 @@ sage_status_t sage_attn_fwd_kres(const void *q, const int64_t q_stride[4], const
     uint16_t *bmean = reinterpret_cast<uint16_t *>(base + cb + sb);
     float *eslot = reinterpret_cast<float *>(base + cb + sb + mb);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_qpass(s, &qs, nullptr, &vs, ws, nullptr, c, st);
-    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
-    if ((e = launch_kres(s, ks, c.k_i8, c.k_scale, bmean, st)) != cudaSuccess)
-        return cuda_fail(e, "K-residual quantization");
+    cudaError_t e = launch_qpass(s, &qs, &ks, &vs, ws, nullptr, c, st, bmean);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass (K-residual mode)");
     if (attn_begin && (e = cudaEventRecord(reinterpret_cast<cudaEvent_t>(attn_begin), st)) != cudaSuccess)
         return cuda_fail(e, "cudaEventRecord");
     if ((e = launch_attention_kres(s, c, qs, bmean, dst(out, o_stride), sm_scale, eslot, n_slots, st)) != cudaSuccess)

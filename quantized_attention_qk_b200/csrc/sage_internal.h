@@ -86,9 +86,11 @@ Codes carve_codes(void *base, const Shape &s);
 // The quantize pass (sage_quant.cu) in one cooperatively launched kernel:
 // statistics of k and/or v, then the codes of the tensors given (null ones are
 // skipped; the combinations q+k+v, q+k, k+v, v and q+v).  `user_k_mean` may be
-// null; the V scales go to c.v_scale.
+// null; the V scales go to c.v_scale.  With `k_bmean` (bf16 [BH][N_pad/64][d])
+// K is coded in K-residual mode instead (combinations q+k+v and k only): the
+// residual of each 64-token block's mean, whose bf16 value goes to k_bmean.
 cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                         float *user_k_mean, const Codes &c, cudaStream_t st);
+                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean = nullptr);
 // 4-D tiled TMA map of a bf16 [B,H,N,d] view: box = 64 channels x `rows` tokens
 // of one (b,h).  The N and H dimensions are handed to the hardware in stride
 // order; *hn_swapped tells the kernel which coordinate comes second.
@@ -130,13 +132,11 @@ cudaError_t launch_attention_sparse(const Shape &s, const Codes &c, const Dst &o
 // (c.q_i8 / c.q_scale are not used).
 cudaError_t launch_attention_fused_q(const Shape &s, const Codes &c, const Src &q_bf16, const Dst &out,
                                      float sm_scale, cudaStream_t st);
-// K-residual mode: the residual codes and bf16 block means (sage_kres.cu),
-// and the attention kernel that computes the mean term (q . mean_b) in its
-// prologue on the tensor cores from the bf16 Q rows and the block means,
-// keeping it in per-SM scratch slots of kres_slots() x nkb x 256 floats
-// (sage_attn.cu).  kres_slots() is the current device's SM count (0 on error).
-cudaError_t launch_kres(const Shape &s, const Src &k, int8_t *k_i8, float *k_scale, uint16_t *k_bmean,
-                        cudaStream_t st);
+// K-residual mode: the attention kernel that computes the mean term
+// (q . mean_b) in its prologue on the tensor cores from the bf16 Q rows and
+// the block means, keeping it in per-SM scratch slots of kres_slots() x nkb x
+// 256 floats (sage_attn.cu).  kres_slots() is the current device's SM count
+// (0 on error).  The residual codes and block means come from launch_qpass.
 int kres_slots();
 cudaError_t launch_attention_kres(const Shape &s, const Codes &c, const Src &q_bf16, const uint16_t *k_bmean,
                                   const Dst &out, float sm_scale, float *eslot, int n_slots, cudaStream_t st);

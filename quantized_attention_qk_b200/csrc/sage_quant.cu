@@ -28,10 +28,20 @@
 //      the codes of Q and K; the attention kernel reads it as an MN-major
 //      operand).
 // Warps work on their own rows and exchange block maxima only within their
-// group; the only CTA-wide barriers are at head boundaries.  The fp64 K sums are exact for bf16 inputs whenever a column's
+// group; the only CTA-wide barriers are at head boundaries.
+//
+// K-residual mode ("ComfyUI-sol-attn", 核心亮点 item 1: quantize only the
+// residual of K inside each block and keep the block-mean term at bf16
+// precision).  Readings where the page is silent: the blocks are the 64-token
+// K blocks; the block mean is the mean of the block's valid tokens (summed
+// exactly in fp64), rounded to bf16 (RNE); the residual fp32(k) - fp32(mean)
+// is coded like the other INT8 codes.  Phase A then sums no K; phase B writes
+// the residual codes, the per-block scales and the bf16 block means (blocks
+// past N: mean 0, codes 0).  The attention kernel adds the mean term.  The fp64 K sums are exact for bf16 inputs whenever a column's
 // values span fewer than 53 bits, so the mean does not depend on how the rows
 // were split among CTAs and warps.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -153,21 +163,29 @@ struct PassArgs {
     unsigned long long *flags;  // [slots]
     unsigned long long stamp;   // 48 bits, bit 47 set
     float *user_k_mean;         // optional copy of the K mean [BH][D]
+    uint16_t *k_bmean;          // K-residual mode: bf16 block means [BH][N_pad/64][D]
     Codes c;
     unsigned *err;
 };
 
-template <int D, bool DO_Q, bool DO_K, bool DO_V>
+// RES: K is coded as the residual of its 64-token block mean (K-residual
+// mode) instead of smoothing by the head's mean, so phase A sums no K.
+template <int D, bool DO_Q, bool DO_K, bool DO_V, bool RES>
 __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
     using Gm = Geom<D>;
     constexpr int VPR = Gm::VPR, RPI = Gm::RPI, NB = Gm::NB, RB = Gm::RB, WU = Gm::WU, KW = Gm::KW, NA = Gm::NA,
                   RA = Gm::RA;
     constexpr int NW = kPassWarps;
-    constexpr bool STATS = DO_K || DO_V;
+    constexpr bool KSUM = DO_K && !RES;  // the head's K column sums (smoothing)
+    constexpr bool STATS = KSUM || DO_V;
     __shared__ double red_s[NW][D];
     __shared__ float red_m[NW][D];
     __shared__ float mu[D], vinv[D];
     __shared__ float grp_max[Gm::GROUPS][2][2][WU];  // [group][unit parity][Q, K][warp]
+    // K-residual mode: the warps' K block sums [group][warp][channel].  One
+    // buffer is enough: between a block's reads and the next block's writes
+    // every warp of the group passes the K-maximum barrier of the block.
+    __shared__ double grp_sum[RES ? Gm::GROUPS : 1][RES ? WU : 1][RES ? D : 1];
     __shared__ AbortState abort_st;
     __shared__ int bad;
     const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock, nsb = (a.N + kKBlock - 1) / kKBlock;
@@ -203,12 +221,12 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
             for (int e = 0; e < 8; ++e) s8[e] = 0.0;
             for (int bt = warp; bt < nbat; bt += NW) {
                 const int rb = r_begin + bt * RA + rl;
-                uint4 kx[DO_K ? NA : 1], vx[DO_V ? NA : 1];
-                if constexpr (DO_K) load_rows<NA, RPI>(kx, kp, a.k.sn, rb, r_end, keep);
+                uint4 kx[KSUM ? NA : 1], vx[DO_V ? NA : 1];
+                if constexpr (KSUM) load_rows<NA, RPI>(kx, kp, a.k.sn, rb, r_end, keep);
                 if constexpr (DO_V) load_rows<NA, RPI>(vx, vp, a.v.sn, rb, r_end, keep);
 #pragma unroll
                 for (int i = 0; i < NA; ++i) {
-                    if (DO_K) {
+                    if constexpr (KSUM) {
                         float f[8];
                         unpack8(kx[i], f);
 #pragma unroll
@@ -249,7 +267,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
                     ss = __dadd_rn(ss, red_s[w][c]);
                     mm = fmaxf(mm, red_m[w][c]);
                 }
-                if (DO_K) a.ksum_part[(int64_t)slot * D + c] = ss;
+                if (KSUM) a.ksum_part[(int64_t)slot * D + c] = ss;
                 if (DO_V) a.vmax_part[(int64_t)slot * D + c] = mm;
             }
             __syncthreads();  // every partial is written (and red_* free again)
@@ -300,14 +318,14 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
                 float mx = 0.f;
                 for (int i = i0; i <= i1; ++i) {
                     const int64_t o = (int64_t)(i + h) * D + c;
-                    if (DO_K) sum = __dadd_rn(sum, __ldcg(a.ksum_part + o));
+                    if (KSUM) sum = __dadd_rn(sum, __ldcg(a.ksum_part + o));
                     if (DO_V) mx = fmaxf(mx, __ldcg(a.vmax_part + o));
                 }
                 const float m = __double2float_rn(__ddiv_rn(sum, static_cast<double>(a.N)));
                 mu[c] = m;
                 vinv[c] = mx > 0.f ? 448.f / mx : 0.f;
                 if (c0 == 0) {  // one CTA writes the per-head outputs
-                    if (DO_K && a.user_k_mean) a.user_k_mean[(int64_t)h * D + c] = m;
+                    if (KSUM && a.user_k_mean) a.user_k_mean[(int64_t)h * D + c] = m;
                     if (DO_V) a.c.v_scale[(int64_t)h * D + c] = mx > 0.f ? mx / 448.f : 0.f;
                 }
             }
@@ -348,9 +366,64 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
             if constexpr (DO_K) {
                 // the warp's rows lie in one 64-token K block, shared by KW warps
                 const uint4 *x = xk;
+                const int kb = (u * kQBlock + gw * RB) / kKBlock;
                 float mu8[8];
+                if constexpr (RES) {
+                    // the block's mean: fp64 sum of its valid rows (exact for
+                    // bf16 inputs), over the KW warps in order, one IEEE
+                    // division, rounded to bf16
+                    double s8[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) mu8[e] = mu[vec * 8 + e];
+                    for (int e = 0; e < 8; ++e) s8[e] = 0.0;
+#pragma unroll
+                    for (int i = 0; i < NB; ++i) {
+                        if (rbase + i * RPI < a.N) {
+                            float f[8];
+                            unpack8(x[i], f);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) s8[e] = __dadd_rn(s8[e], static_cast<double>(f[e]));
+                        }
+                    }
+#pragma unroll
+                    for (int o = VPR; o < 32; o <<= 1) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) s8[e] = __dadd_rn(s8[e], __shfl_xor_sync(0xffffffffu, s8[e], o));
+                    }
+                    if (KW > 1) {
+                        if (lane < VPR) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) grp_sum[grp][gw][vec * 8 + e] = s8[e];
+                        }
+                        group_sync(1 + grp, 32 * WU);
+                        const int w0 = gw - gw % KW;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            double t = 0.0;
+#pragma unroll
+                            for (int w = 0; w < KW; ++w) t = __dadd_rn(t, grp_sum[grp][w0 + w][vec * 8 + e]);
+                            s8[e] = t;
+                        }
+                    }
+                    const int nvalid = max(0, min(kKBlock, a.N - kb * kKBlock));
+                    uint32_t mw[4];
+#pragma unroll
+                    for (int e = 0; e < 8; e += 2) {
+                        const __nv_bfloat16 m0 =
+                            __double2bfloat16(nvalid > 0 ? __ddiv_rn(s8[e], static_cast<double>(nvalid)) : 0.0);
+                        const __nv_bfloat16 m1 =
+                            __double2bfloat16(nvalid > 0 ? __ddiv_rn(s8[e + 1], static_cast<double>(nvalid)) : 0.0);
+                        mu8[e] = __bfloat162float(m0);
+                        mu8[e + 1] = __bfloat162float(m1);
+                        mw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(m0)) |
+                                    (static_cast<uint32_t>(__bfloat16_as_ushort(m1)) << 16);
+                    }
+                    if (gw % KW == 0 && lane < VPR)
+                        *reinterpret_cast<uint4 *>(a.k_bmean + ((int64_t)h * nkb + kb) * D + vec * 8) =
+                            make_uint4(mw[0], mw[1], mw[2], mw[3]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) mu8[e] = mu[vec * 8 + e];
+                }
                 float ka = 0.f;
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
@@ -386,8 +459,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
                     }
                     *reinterpret_cast<uint2 *>(a.c.k_i8 + obase + (int64_t)i * RPI * D) = i8x8(d, inv);
                 }
-                if (gw % KW == 0 && lane == 0)
-                    a.c.k_scale[(int64_t)h * nkb + (u * kQBlock + gw * RB) / kKBlock] = ka > 0.f ? ka / 127.f : 0.f;
+                if (gw % KW == 0 && lane == 0) a.c.k_scale[(int64_t)h * nkb + kb] = ka > 0.f ? ka / 127.f : 0.f;
             }
             if constexpr (DO_V) {
                 const uint4 *x = xv;
@@ -416,9 +488,9 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
     }
 }
 
-template <int D, bool DQ, bool DK, bool DV>
+template <int D, bool DQ, bool DK, bool DV, bool RES = false>
 cudaError_t launch_qpass_k(const Shape &s, const PassArgs &a, cudaStream_t st) {
-    auto kern = k_qpass<D, DQ, DK, DV>;
+    auto kern = k_qpass<D, DQ, DK, DV, RES>;
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -454,7 +526,7 @@ unsigned long long next_stamp() {
 
 template <int D>
 cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                           float *user_k_mean, const Codes &c, cudaStream_t st) {
+                           float *user_k_mean, const Codes &c, uint16_t *k_bmean, cudaStream_t st) {
     PassArgs a{};
     const Src none{nullptr, 0, 0, 0};
     a.q = q ? *q : none;
@@ -469,8 +541,14 @@ cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src
     a.flags = ws.flags;
     a.stamp = next_stamp();
     a.user_k_mean = user_k_mean;
+    a.k_bmean = k_bmean;
     a.c = c;
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
+    if (k_bmean) {  // K-residual mode
+        if (q && k && v) return launch_qpass_k<D, true, true, true, true>(s, a, st);
+        if (!q && k && !v) return launch_qpass_k<D, false, true, false, true>(s, a, st);
+        return cudaErrorInvalidValue;
+    }
     if (q && k && v) return launch_qpass_k<D, true, true, true>(s, a, st);
     if (q && k && !v) return launch_qpass_k<D, true, true, false>(s, a, st);
     if (!q && k && v) return launch_qpass_k<D, false, true, true>(s, a, st);
@@ -482,9 +560,9 @@ cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src
 }  // namespace
 
 cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                         float *user_k_mean, const Codes &c, cudaStream_t st) {
-    return s.d == 128 ? launch_qpass_d<128>(s, q, k, v, ws, user_k_mean, c, st)
-                      : launch_qpass_d<64>(s, q, k, v, ws, user_k_mean, c, st);
+                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean) {
+    return s.d == 128 ? launch_qpass_d<128>(s, q, k, v, ws, user_k_mean, c, k_bmean, st)
+                      : launch_qpass_d<64>(s, q, k, v, ws, user_k_mean, c, k_bmean, st);
 }
 
 }  // namespace sage
