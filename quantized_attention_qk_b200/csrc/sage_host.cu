@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <mutex>
+#include <vector>
 
 #include "sage.h"
 #include "sage_internal.h"
@@ -19,6 +20,7 @@ constexpr size_t kAlign = 1024;
 size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 constexpr int kStreams = 3;  // internal streams (and chunk workspaces)
+constexpr int kTailSplits = 2;  // the call's last chunk is cut into up to 3 halving pieces
 
 // Heads per chunk: about 64 MiB of input per chunk, between 4 and 16 chunks
 // per call (small chunks make the strided copies of a fused layout slow; few
@@ -172,10 +174,27 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
     uint16_t *h_out = static_cast<uint16_t *>(out_host);
     const int64_t hd = (int64_t)H * d, nd = (int64_t)N * d;
 
-    int c = 0;  // chunk count: chunk c runs on stream c % kStreams with that stream's workspace
+    // the chunks: hc_max heads each, the last one of the call cut into
+    // halving pieces (e.g. 6 heads -> 3, 2, 1), so that what cannot overlap
+    // anything -- the last chunk's kernels and copy back -- is short
+    struct Chunk { int b, h0, hc; };
+    std::vector<Chunk> plan;
     for (int b = 0; b < B; ++b)
-        for (int h0 = 0; h0 < H; h0 += hc_max, ++c) {
-            const int hc = H - h0 < hc_max ? H - h0 : hc_max;
+        for (int h0 = 0; h0 < H; h0 += hc_max) plan.push_back({b, h0, H - h0 < hc_max ? H - h0 : hc_max});
+    {
+        const Chunk last = plan.back();
+        plan.pop_back();
+        int h0 = last.h0, rem = last.hc;
+        for (int i = 0; i < kTailSplits && rem > 1; ++i) {
+            const int half = (rem + 1) / 2;
+            plan.push_back({last.b, h0, half});
+            h0 += half;
+            rem -= half;
+        }
+        if (rem > 0) plan.push_back({last.b, h0, rem});
+    }
+    for (int c = 0; c < static_cast<int>(plan.size()); ++c) {
+            const int b = plan[c].b, h0 = plan[c].h0, hc = plan[c].hc;
             cudaStream_t s = st[c % kStreams];
             char *ws = ws0 + (c % kStreams) * ws_step;
             const Shape cs{1, hc, N, d};
