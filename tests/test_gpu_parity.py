@@ -69,7 +69,22 @@ def _check_attn(w, heads=None, nrows=None, seed=0):
 def test_quant_codes_match_oracle(name, hs):
     """Every code and scale of the quantize pass equals the oracle's bit for
     bit, the K mean included (heads hs, counted over b*H + h)."""
-    w = WORKLOADS[name]
+    _check_quant(WORKLOADS[name], hs)
+
+
+@pytest.mark.parametrize("B,H,N,d", [(8, 64, 100, 64), (2, 300, 130, 128), (1, 3, 20000, 64), (3, 1, 4097, 128)])
+def test_quant_codes_match_oracle_on_many_heads_and_ragged_lengths(B, H, N, d):
+    """The quantize kernel splits all heads' rows evenly over its CTAs, so
+    with many short heads a CTA covers several heads in both of its phases,
+    and with few long ones many CTAs share a head's statistics; every head's
+    codes and scales must still equal the oracle's bit for bit."""
+    w = tiny_custom(B, H, N, d, seed=1201 + N, bias_sigma=2.0, outlier_frac=0.02)
+    hs = list(range(B * H)) if B * H <= 8 else [0, 1, B * H // 2, B * H - 2, B * H - 1]
+    _check_quant(w, hs)
+
+
+def _check_quant(w, hs):
+    name = w.name
     (q, k, v), (qd, kd, vd), _ = _inputs(w)
     r = sage.sage_quant_qk(qd, kd)
     v_e4m3, v_scale = sage.sage_quant_v(vd)
