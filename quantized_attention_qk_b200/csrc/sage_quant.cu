@@ -28,7 +28,10 @@
 //      the codes of Q and K; the attention kernel reads it as an MN-major
 //      operand).
 // Warps work on their own rows and exchange block maxima only within their
-// group; the only CTA-wide barriers are at head boundaries.
+// group; the only CTA-wide barriers are at head boundaries.  The fp64 K sums
+// are exact for bf16 inputs whenever a column's values span fewer than 53
+// bits, so the mean does not depend on how the rows were split among CTAs and
+// warps.
 //
 // K-residual mode ("ComfyUI-sol-attn", 核心亮点 item 1: quantize only the
 // residual of K inside each block and keep the block-mean term at bf16
@@ -37,9 +40,7 @@
 // exactly in fp64), rounded to bf16 (RNE); the residual fp32(k) - fp32(mean)
 // is coded like the other INT8 codes.  Phase A then sums no K; phase B writes
 // the residual codes, the per-block scales and the bf16 block means (blocks
-// past N: mean 0, codes 0).  The attention kernel adds the mean term.  The fp64 K sums are exact for bf16 inputs whenever a column's
-// values span fewer than 53 bits, so the mean does not depend on how the rows
-// were split among CTAs and warps.
+// past N: mean 0, codes 0).  The attention kernel adds the mean term.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
