@@ -432,7 +432,9 @@ def run_gpu(args):
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
                        "attention, bf16 out -> pinned host; dense)"},
-        "gpu_launches": (LAUNCHES_PER_STEP + (3 if args.tau is not None and args.tau < 1 else 0)) * args.steps,
+        # a selecting forward adds the selection's scoring and ranking kernels
+        # (the quantize pass pools the tiles itself)
+        "gpu_launches": (LAUNCHES_PER_STEP + (2 if args.tau is not None and args.tau < 1 else 0)) * args.steps,
         "clocks": r["clocks"],
     }
     if args.tau is not None:

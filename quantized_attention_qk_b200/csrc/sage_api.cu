@@ -393,16 +393,20 @@ sage_status_t sage_attn_fwd_sparse(const void *q, const int64_t q_stride[4], con
     const Codes c = carve_codes(base, s);
     const StatsWs ws = carve_stats_ws(base + cb, s);
     const Src qs = src(q, q_stride), ks = src(k, k_stride), vs = src(v, v_stride);
-    cudaError_t e = launch_qpass(s, &qs, &ks, &vs, ws, nullptr, c, st);
-    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     // tau >= 1 keeps every key tile (reading S3): the dense kernel computes the
     // same result bit for bit without walking step lists
     const bool dense = !mask_in && tau >= 1.f;
+    const bool select = !mask_in && (!dense || mask_out);
+    // with a selection to run, the quantize pass also pools the tiles' codes
+    float *pool_qv = nullptr, *pool_kvT = nullptr;
+    if (select) select_pool_ptrs(base + cb + sb, s, &pool_qv, &pool_kvT);
+    cudaError_t e = launch_qpass(s, &qs, &ks, &vs, ws, nullptr, c, st, nullptr, pool_qv, pool_kvT);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize pass");
     const uint32_t *mask = mask_in;
-    if (!mask && (!dense || mask_out)) {
+    if (select) {
         uint32_t *m = mask_out ? mask_out : reinterpret_cast<uint32_t *>(base + cb + sb + selb);
         if ((e = launch_select(s, c.q_i8, c.q_scale, c.k_i8, c.k_scale, sm_scale, tau, base + cb + sb, m, nullptr,
-                               st)) != cudaSuccess)
+                               st, true)) != cudaSuccess)
             return cuda_fail(e, "block selection");
         mask = m;
     } else if (mask_out) {

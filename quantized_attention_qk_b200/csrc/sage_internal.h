@@ -89,8 +89,12 @@ Codes carve_codes(void *base, const Shape &s);
 // null; the V scales go to c.v_scale.  With `k_bmean` (bf16 [BH][N_pad/64][d])
 // K is coded in K-residual mode instead (combinations q+k+v and k only): the
 // residual of each 64-token block's mean, whose bf16 value goes to k_bmean.
+// With pool_qv / pool_kvT (q+k+v, smoothing) it also writes the pooled tile
+// vectors of the block selection (select_pool_ptrs), so that launch_select
+// can skip its pooling kernel.
 cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean = nullptr);
+                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean = nullptr,
+                         float *pool_qv = nullptr, float *pool_kvT = nullptr);
 // 4-D tiled TMA map of a bf16 [B,H,N,d] view: box = 64 channels x `rows` tokens
 // of one (b,h).  The N and H dimensions are handed to the hardware in stride
 // order; *hn_swapped tells the kernel which coordinate comes second.
@@ -145,12 +149,16 @@ cudaError_t launch_debug_qk_tile(const Shape &s, const int8_t *q_i8, const int8_
 cudaError_t read_and_clear_device_error(unsigned *value, cudaStream_t st);
 
 // Block-sparse selection (sage_sparse.cu): scratch for the pooled tile
-// vectors, the mask size, and the launcher (scores, ranking, kept prefix).
+// vectors, the mask size, and the launcher (pooling, scores, ranking, kept
+// prefix).  select_pool_ptrs gives the pooled vectors' places in that
+// scratch; with `pooled` the launcher takes them as already written there
+// (by the quantize pass) and skips its pooling kernel.
 size_t select_ws_bytes(const Shape &s);
 size_t mask_bytes(const Shape &s);
+void select_pool_ptrs(void *ws, const Shape &s, float **qv, float **kvT);
 cudaError_t launch_select(const Shape &s, const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
                           const float *k_scale, float sm_scale, float tau, void *ws, uint32_t *mask, float *sbar_out,
-                          cudaStream_t st);
+                          cudaStream_t st, bool pooled = false);
 
 // Dense fp32 reference (sage_dense_ref.cu).
 cudaError_t launch_dense_ref(const Shape &s, const Src &q, const Src &k, const Src &v, const Dst &out,

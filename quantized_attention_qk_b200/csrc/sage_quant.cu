@@ -150,6 +150,33 @@ __device__ __forceinline__ void load_rows(uint4 (&x)[NV], const uint16_t *p, int
     }
 }
 
+// Tile pooling: add 8 int8 codes (channels 0..7 of this lane's vector) into
+// four int16 pairs (channels 2j, 2j+1 in pair j), sign-extending each byte.
+__device__ __forceinline__ uint32_t sext_pair(uint32_t w, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));  // selector bit 3: replicate the byte's sign
+    return r;
+}
+__device__ __forceinline__ void add_codes(uint32_t (&ps)[4], uint2 cw) {
+    ps[0] = __vadd2(ps[0], sext_pair(cw.x, 0x9180u));
+    ps[1] = __vadd2(ps[1], sext_pair(cw.x, 0xB3A2u));
+    ps[2] = __vadd2(ps[2], sext_pair(cw.y, 0x9180u));
+    ps[3] = __vadd2(ps[3], sext_pair(cw.y, 0xB3A2u));
+}
+// The warp's sums: lanes VPR apart hold the same channels; lanes < VPR store
+// theirs into the warp's slot (D/2 int16 pairs).
+template <int VPR>
+__device__ __forceinline__ void pool_partial(uint32_t (&ps)[4], uint32_t *slot, int lane, int vec) {
+#pragma unroll
+    for (int o = VPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ps[j] = __vadd2(ps[j], __shfl_xor_sync(0xffffffffu, ps[j], o));
+    if (lane < VPR) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) slot[vec * 4 + j] = ps[j];
+    }
+}
+
 // A flag of phase A holds (stamp << 16) | readers: the call's 48-bit stamp
 // and the number of phase-B CTAs that read the head (known from the split).
 // Each reader takes one off after its wait and the last one clears the flag,
@@ -165,13 +192,16 @@ struct PassArgs {
     unsigned long long stamp;   // 48 bits, bit 47 set
     float *user_k_mean;         // optional copy of the K mean [BH][D]
     uint16_t *k_bmean;          // K-residual mode: bf16 block means [BH][N_pad/64][D]
+    float *pool_qv, *pool_kvT;  // tile pooling: [BH][tiles][D] and [BH][D][tiles]
     Codes c;
     unsigned *err;
 };
 
 // RES: K is coded as the residual of its 64-token block mean (K-residual
 // mode) instead of smoothing by the head's mean, so phase A sums no K.
-template <int D, bool DO_Q, bool DO_K, bool DO_V, bool RES>
+// POOL: also the pooled tile vectors of the block selection (the code sums
+// of each 128-token tile, times the scales), from the codes in registers.
+template <int D, bool DO_Q, bool DO_K, bool DO_V, bool RES, bool POOL = false>
 __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
     using Gm = Geom<D>;
     constexpr int VPR = Gm::VPR, RPI = Gm::RPI, NB = Gm::NB, RB = Gm::RB, WU = Gm::WU, KW = Gm::KW, NA = Gm::NA,
@@ -187,6 +217,10 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
     // buffer is enough: between a block's reads and the next block's writes
     // every warp of the group passes the K-maximum barrier of the block.
     __shared__ double grp_sum[RES ? Gm::GROUPS : 1][RES ? WU : 1][RES ? D : 1];
+    // tile pooling: the warps' code sums as int16 pairs [group][Q, K][warp][channel pair],
+    // and the amax of the unit's two K blocks
+    __shared__ uint32_t grp_pool[POOL ? Gm::GROUPS : 1][2][POOL ? WU : 1][POOL ? D / 2 : 1];
+    __shared__ float grp_ka[POOL ? Gm::GROUPS : 1][2];
     __shared__ AbortState abort_st;
     __shared__ int bad;
     const int nqb = a.n_pad / kQBlock, nkb = a.n_pad / kKBlock, nsb = (a.N + kKBlock - 1) / kKBlock;
@@ -336,6 +370,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
         for (int u = c1 - 1 - grp; u >= c0; u -= Gm::GROUPS) {
             const int rbase = u * kQBlock + gw * RB + rl;  // this lane's first row
             const int64_t obase = ((int64_t)h * a.n_pad + rbase) * D + vec * 8;
+            float q_scale_unit = 0.f;  // POOL: the block's Q scale
             // all of the block's rows are requested at once: one memory latency per block
             uint4 xq[DO_Q ? NB : 1], xk[DO_K ? NB : 1], xv[DO_V ? NB : 1];
             if constexpr (DO_Q) load_rows<NB, RPI>(xq, a.q.p + b * a.q.sb + hh * a.q.sh + vec * 8, a.q.sn, rbase, a.N, drop);
@@ -356,13 +391,18 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
 #pragma unroll
                 for (int w = 0; w < WU; ++w) qa = fmaxf(qa, grp_max[grp][parity][0][w]);
                 const float inv = qa > 0.f ? 127.f / qa : 0.f;
+                uint32_t ps[4] = {0u, 0u, 0u, 0u};  // POOL: this lane's code sums per channel, int16 pairs
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
                     float f[8];
                     unpack8(x[i], f);
-                    *reinterpret_cast<uint2 *>(a.c.q_i8 + obase + (int64_t)i * RPI * D) = i8x8(f, inv);
+                    const uint2 cw = i8x8(f, inv);
+                    *reinterpret_cast<uint2 *>(a.c.q_i8 + obase + (int64_t)i * RPI * D) = cw;
+                    if constexpr (POOL) add_codes(ps, cw);
                 }
-                if (gw == 0 && lane == 0) a.c.q_scale[(int64_t)h * nqb + u] = qa > 0.f ? qa / 127.f : 0.f;
+                if constexpr (POOL) pool_partial<VPR>(ps, grp_pool[grp][0][gw], lane, vec);
+                q_scale_unit = qa > 0.f ? qa / 127.f : 0.f;
+                if (gw == 0 && lane == 0) a.c.q_scale[(int64_t)h * nqb + u] = q_scale_unit;
             }
             if constexpr (DO_K) {
                 // the warp's rows lie in one 64-token K block, shared by KW warps
@@ -446,6 +486,7 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
                     for (int w = 0; w < KW; ++w) ka = fmaxf(ka, grp_max[grp][parity][1][w0 + w]);
                 }
                 const float inv = ka > 0.f ? 127.f / ka : 0.f;
+                uint32_t ps[4] = {0u, 0u, 0u, 0u};  // POOL: this lane's code sums per channel, int16 pairs
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
                     float d[8];
@@ -458,9 +499,43 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
 #pragma unroll
                         for (int e = 0; e < 8; ++e) d[e] = 0.f;
                     }
-                    *reinterpret_cast<uint2 *>(a.c.k_i8 + obase + (int64_t)i * RPI * D) = i8x8(d, inv);
+                    const uint2 cw = i8x8(d, inv);
+                    *reinterpret_cast<uint2 *>(a.c.k_i8 + obase + (int64_t)i * RPI * D) = cw;
+                    if constexpr (POOL) add_codes(ps, cw);
                 }
                 if (gw % KW == 0 && lane == 0) a.c.k_scale[(int64_t)h * nkb + kb] = ka > 0.f ? ka / 127.f : 0.f;
+                if constexpr (POOL) {
+                    pool_partial<VPR>(ps, grp_pool[grp][1][gw], lane, vec);
+                    if (gw % KW == 0 && lane == 0) grp_ka[grp][gw / KW] = ka;
+                    // the tile's pooled vectors (the code sums are exact in int16:
+                    // at most 128 rows of |code| <= 127): qv = q_scale * sum of the Q
+                    // codes, kvT = k_scale(2u) * sum of K block 2u + (the second block
+                    // only if it holds a token) k_scale(2u+1) * its sum, one rounding
+                    // per operation
+                    group_sync(1 + grp, 32 * WU);
+                    for (int t = gw * 32 + lane; t < D / 2; t += 32 * WU) {
+                        uint32_t sq = 0u, s0 = 0u, s1 = 0u;
+#pragma unroll
+                        for (int w = 0; w < WU; ++w) {
+                            sq = __vadd2(sq, grp_pool[grp][0][w][t]);
+                            if (w < KW) s0 = __vadd2(s0, grp_pool[grp][1][w][t]);
+                            else s1 = __vadd2(s1, grp_pool[grp][1][w][t]);
+                        }
+                        const float ks0 = grp_ka[grp][0] > 0.f ? grp_ka[grp][0] / 127.f : 0.f;
+                        const float ks1 = grp_ka[grp][1] > 0.f ? grp_ka[grp][1] / 127.f : 0.f;
+                        const bool second = (2 * u + 1) * kKBlock < a.N;
+#pragma unroll
+                        for (int hf = 0; hf < 2; ++hf) {
+                            const int c = 2 * t + hf;
+                            const float fq = static_cast<float>(static_cast<int16_t>(sq >> (16 * hf)));
+                            const float f0 = static_cast<float>(static_cast<int16_t>(s0 >> (16 * hf)));
+                            const float f1 = static_cast<float>(static_cast<int16_t>(s1 >> (16 * hf)));
+                            a.pool_qv[((int64_t)h * nqb + u) * D + c] = __fmul_rn(q_scale_unit, fq);
+                            const float k1 = second ? __fmul_rn(ks1, f1) : 0.f;
+                            a.pool_kvT[((int64_t)h * D + c) * nqb + u] = __fadd_rn(__fmul_rn(ks0, f0), k1);
+                        }
+                    }
+                }
             }
             if constexpr (DO_V) {
                 const uint4 *x = xv;
@@ -489,9 +564,9 @@ __global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
     }
 }
 
-template <int D, bool DQ, bool DK, bool DV, bool RES = false>
+template <int D, bool DQ, bool DK, bool DV, bool RES = false, bool POOL = false>
 cudaError_t launch_qpass_k(const Shape &s, const PassArgs &a, cudaStream_t st) {
-    auto kern = k_qpass<D, DQ, DK, DV, RES>;
+    auto kern = k_qpass<D, DQ, DK, DV, RES, POOL>;
     int dev = 0, sms = 0, per_sm = 0;
     cudaError_t e;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
@@ -527,7 +602,8 @@ unsigned long long next_stamp() {
 
 template <int D>
 cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                           float *user_k_mean, const Codes &c, uint16_t *k_bmean, cudaStream_t st) {
+                           float *user_k_mean, const Codes &c, uint16_t *k_bmean, float *pool_qv, float *pool_kvT,
+                           cudaStream_t st) {
     PassArgs a{};
     const Src none{nullptr, 0, 0, 0};
     a.q = q ? *q : none;
@@ -543,8 +619,14 @@ cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src
     a.stamp = next_stamp();
     a.user_k_mean = user_k_mean;
     a.k_bmean = k_bmean;
+    a.pool_qv = pool_qv;
+    a.pool_kvT = pool_kvT;
     a.c = c;
     if (!(a.err = device_error_ptr())) return cudaErrorSymbolNotFound;
+    if (pool_qv || pool_kvT) {  // with the pooled tile vectors of the block selection
+        if (q && k && v && !k_bmean && pool_qv && pool_kvT) return launch_qpass_k<D, true, true, true, false, true>(s, a, st);
+        return cudaErrorInvalidValue;
+    }
     if (k_bmean) {  // K-residual mode
         if (q && k && v) return launch_qpass_k<D, true, true, true, true>(s, a, st);
         if (!q && k && !v) return launch_qpass_k<D, false, true, false, true>(s, a, st);
@@ -561,9 +643,10 @@ cudaError_t launch_qpass_d(const Shape &s, const Src *q, const Src *k, const Src
 }  // namespace
 
 cudaError_t launch_qpass(const Shape &s, const Src *q, const Src *k, const Src *v, const StatsWs &ws,
-                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean) {
-    return s.d == 128 ? launch_qpass_d<128>(s, q, k, v, ws, user_k_mean, c, k_bmean, st)
-                      : launch_qpass_d<64>(s, q, k, v, ws, user_k_mean, c, k_bmean, st);
+                         float *user_k_mean, const Codes &c, cudaStream_t st, uint16_t *k_bmean, float *pool_qv,
+                         float *pool_kvT) {
+    return s.d == 128 ? launch_qpass_d<128>(s, q, k, v, ws, user_k_mean, c, k_bmean, pool_qv, pool_kvT, st)
+                      : launch_qpass_d<64>(s, q, k, v, ws, user_k_mean, c, k_bmean, pool_qv, pool_kvT, st);
 }
 
 }  // namespace sage

@@ -221,27 +221,36 @@ size_t select_ws_bytes(const Shape &s) {
 
 size_t mask_bytes(const Shape &s) { return (size_t)s.BH() * s.n_tiles() * s.mask_words() * sizeof(uint32_t); }
 
+void select_pool_ptrs(void *ws, const Shape &s, float **qv, float **kvT) {
+    char *w = static_cast<char *>(ws);
+    const size_t vec = up((size_t)s.BH() * s.n_tiles() * s.d * sizeof(float));
+    *qv = reinterpret_cast<float *>(w);
+    *kvT = reinterpret_cast<float *>(w + vec);
+}
+
 cudaError_t launch_select(const Shape &s, const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
                           const float *k_scale, float sm_scale, float tau, void *ws, uint32_t *mask, float *sbar_out,
-                          cudaStream_t st) {
+                          cudaStream_t st, bool pooled) {
     const int nt = s.n_tiles();
     if (nt > kMaxSelectTiles) return cudaErrorInvalidValue;
     char *w = static_cast<char *>(ws);
     const size_t vec = up((size_t)s.BH() * nt * s.d * sizeof(float));
-    float *qv = reinterpret_cast<float *>(w);
-    float *kvT = reinterpret_cast<float *>(w + vec);
+    float *qv = nullptr, *kvT = nullptr;
+    select_pool_ptrs(ws, s, &qv, &kvT);
     float *sbar = sbar_out ? sbar_out : reinterpret_cast<float *>(w + 2 * vec);
     const float s_l2 = sm_scale * static_cast<float>(1.4426950408889634);
     const int P = pow2_at_least(nt), words = s.mask_words();
     const dim3 g1(nt, s.BH()), g2((nt + kScoreTile - 1) / kScoreTile, (nt + kScoreTile - 1) / kScoreTile, s.BH());
     const size_t smem = (size_t)(2 * P + words) * 4;
     if (s.d == 128) {
-        k_pool<128><<<g1, kPoolThreads, 0, st>>>(q_i8, q_scale, k_i8, k_scale, s.N, s.n_pad(), s.n_qblocks(),
-                                                 s.n_kblocks(), nt, qv, kvT);
+        if (!pooled)
+            k_pool<128><<<g1, kPoolThreads, 0, st>>>(q_i8, q_scale, k_i8, k_scale, s.N, s.n_pad(), s.n_qblocks(),
+                                                     s.n_kblocks(), nt, qv, kvT);
         k_score<128><<<g2, kScoreThreads, 0, st>>>(qv, kvT, s.N, nt, s_l2, sbar);
     } else {
-        k_pool<64><<<g1, kPoolThreads, 0, st>>>(q_i8, q_scale, k_i8, k_scale, s.N, s.n_pad(), s.n_qblocks(),
-                                                s.n_kblocks(), nt, qv, kvT);
+        if (!pooled)
+            k_pool<64><<<g1, kPoolThreads, 0, st>>>(q_i8, q_scale, k_i8, k_scale, s.N, s.n_pad(), s.n_qblocks(),
+                                                    s.n_kblocks(), nt, qv, kvT);
         k_score<64><<<g2, kScoreThreads, 0, st>>>(qv, kvT, s.N, nt, s_l2, sbar);
     }
     k_select<<<g1, kSelThreads, smem, st>>>(sbar, s.N, nt, P, words, tau, mask);

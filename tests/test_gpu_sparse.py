@@ -213,3 +213,20 @@ def test_single_tile_sequences():
     assert torch.count_nonzero(empty).item() == 0
     assert torch.equal(sel, dense)  # one tile: every tau keeps it
     assert sage.mask_to_keep(mask, 1).all()
+
+
+@pytest.mark.parametrize("w", [WORKLOADS["flux"], WORKLOADS["sdxl"], tiny_custom(2, 3, 1000, 128, 561, bias_sigma=3.0)],
+                         ids=lambda w: w.name)
+def test_forward_selection_equals_the_standalone_selection_on_its_codes(w):
+    """The selecting forward pools the tiles' codes inside its quantize pass;
+    sage_block_select pools them from the codes in a kernel of its own.  On
+    the same inputs (whose codes both sides share bit for bit) the two kept
+    sets must be the same on every row, for several tau."""
+    _, dev = _inputs(w, planted=True)
+    codes = sage.sage_quant_qk(dev[0], dev[1])
+    for tau in (0.3, 0.5, 0.9):
+        _, mask = sage.sage_attn_fwd_sparse(*dev, tau=tau, sm_scale=w.sm_scale, return_mask=True)
+        alone = sage.sage_block_select(codes, w.N, w.sm_scale, tau)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        assert torch.equal(mask, alone), (w.name, tau)
