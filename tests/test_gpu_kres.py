@@ -95,3 +95,28 @@ def test_flux_sampled_rows_and_error_against_exact():
     # both schemes sit at their intrinsic error (about 0.05 on this workload)
     assert err_k < 0.08 and err_s < 0.08, (err_k, err_s)
     print(f"flux vs exact: K-residual {err_k:.4f}, smoothing {err_s:.4f}")
+
+
+@pytest.mark.parametrize("name,heads", [("video", [(0, 0), (0, 39)]), ("long64k", [(0, 5)])])
+def test_long_sequences_sampled_rows(name, heads):
+    """Sequences whose K blocks fill more than one of the attention prologue's
+    chunks of 256 block means (video: 532 blocks, three chunks; 65K tokens:
+    1024 blocks, four chunks) against the oracle's K-residual emulation on
+    sampled rows (first, last, tail and random)."""
+    w = WORKLOADS[name]
+    assert -(-w.N // 64) > 256
+    q, k, v, _ = make_qkv(w)
+    qd, kd, vd, _ = make_qkv(w, device=DEV)
+    out = sage.sage_attn_fwd_kres(qd, kd, vd, sm_scale=w.sm_scale)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    rows = U.sample_rows(w.N, 24, 13)
+    got = U.stack(U.gather(out, heads, rows), heads)
+    want = []
+    for (b, h) in heads:
+        sl = (slice(b, b + 1), slice(h, h + 1))
+        _, bits = oracle.attn_quant(q[sl], k[sl], v[sl], w.sm_scale, rows=rows, k_residual=True)
+        want.append(oracle.bf16_bits_to_f64(bits[0, 0]))
+    ok, rel, mx, nstep = U.within_tol(got, np.stack(want), label="K-residual " + name)
+    assert np.isfinite(got).all()
+    assert ok, (name, rel, mx, nstep)
