@@ -55,7 +55,7 @@
 namespace sage {
 namespace {
 
-constexpr int kPassWarps = 16;
+constexpr int kPassWarps = 8;  // two CTAs per SM (128 registers a thread)
 constexpr int kPassThreads = 32 * kPassWarps;
 
 // Geometry of one warp's rows for head dim D: a warp load instruction covers
@@ -202,7 +202,7 @@ struct PassArgs {
 // POOL: also the pooled tile vectors of the block selection (the code sums
 // of each 128-token tile, times the scales), from the codes in registers.
 template <int D, bool DO_Q, bool DO_K, bool DO_V, bool RES, bool POOL = false>
-__global__ void __launch_bounds__(kPassThreads, 1) k_qpass(const PassArgs a) {
+__global__ void __launch_bounds__(kPassThreads, 512 / kPassThreads) k_qpass(const PassArgs a) {
     using Gm = Geom<D>;
     constexpr int VPR = Gm::VPR, RPI = Gm::RPI, NB = Gm::NB, RB = Gm::RB, WU = Gm::WU, KW = Gm::KW, NA = Gm::NA,
                   RA = Gm::RA;
