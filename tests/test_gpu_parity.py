@@ -161,6 +161,19 @@ def test_ragged_and_short_sequences(N, d):
     _check_attn(tiny_custom(1, 1, N, d, seed=7 * N + d, bias_sigma=2.0))
 
 
+@pytest.mark.parametrize("B,H,N,d", [(1, 65535, 1, 64), (5, 13107, 3, 128)])
+def test_the_largest_head_count(B, H, N, d):
+    """B*H at its limit (65535 heads, the attention grid's second dimension)
+    with very short heads: every CTA of the quantize kernel covers hundreds of
+    heads in both of its phases.  Codes, scales and the forward's rows equal
+    the oracle's on heads at the start, the middle and the end."""
+    w = tiny_custom(B, H, N, d, seed=991 + N, bias_sigma=2.0)
+    hs = [0, 1, B * H // 2, B * H - 2, B * H - 1]
+    _check_quant(w, hs)
+    heads = [divmod(x, H) for x in hs]
+    _check_attn(w, heads=heads, nrows=None)
+
+
 def test_batched_heads_d64():
     _check_attn(tiny_custom(3, 2, 200, 64, seed=77, bias_sigma=1.0), nrows=None)
 
