@@ -84,31 +84,36 @@ def test_quant_codes_match_oracle_on_many_heads_and_ragged_lengths(B, H, N, d):
 
 
 def _check_quant(w, hs):
-    name = w.name
     (q, k, v), (qd, kd, vd), _ = _inputs(w)
     r = sage.sage_quant_qk(qd, kd)
     v_e4m3, v_scale = sage.sage_quant_v(vd)
     torch.cuda.synchronize()
     sage.sage_check()
-    N = w.N
-    nqb, nkb = -(-N // 128), -(-N // 64)
     for bh in hs:
         b, h = divmod(bh, w.H)
         sl = (slice(b, b + 1), slice(h, h + 1))
         o = oracle.quantize(q[sl], k[sl], v[sl])
-        for key, n_valid in (("q_i8", N), ("k_i8", N)):
-            g = r[key][b, h].cpu().numpy()
-            np.testing.assert_array_equal(g[:N], o[key][0, 0], err_msg=f"{name} {key} head {bh}")
-            assert (g[N:] == 0).all()
-        np.testing.assert_array_equal(r["q_scale"][b, h, :nqb].cpu().numpy(), o["q_scale"][0, 0])
-        assert (r["q_scale"][b, h, nqb:] == 0).all()
-        np.testing.assert_array_equal(r["k_mean"][b, h].cpu().numpy(), o["k_mean"][0, 0])
-        np.testing.assert_array_equal(r["k_scale"][b, h, :nkb].cpu().numpy(), o["k_scale"][0, 0])
-        assert (r["k_scale"][b, h, nkb:] == 0).all()
-        gv = v_e4m3[b, h].cpu().numpy()          # [N_pad, d]
-        np.testing.assert_array_equal(gv[:N], o["v_e4m3"][0, 0])
-        assert (gv[N:] == 0).all()
-        np.testing.assert_array_equal(v_scale[b, h].cpu().numpy(), o["v_scale"][0, 0])
+        _assert_head_codes(r, v_e4m3, v_scale, b, h, w.N, o, f"{w.name} head {bh}")
+
+
+def _assert_head_codes(r, v_e4m3, v_scale, b, h, N, o, label):
+    """Head (b, h) of the quantize pass's outputs against the oracle's codes
+    of that head alone (o, from oracle.quantize on [1,1,N,d] inputs): every
+    code and scale equal, padded rows and blocks zero."""
+    nqb, nkb = -(-N // 128), -(-N // 64)
+    for key in ("q_i8", "k_i8"):
+        g = r[key][b, h].cpu().numpy()
+        np.testing.assert_array_equal(g[:N], o[key][0, 0], err_msg=f"{label} {key}")
+        assert (g[N:] == 0).all()
+    np.testing.assert_array_equal(r["q_scale"][b, h, :nqb].cpu().numpy(), o["q_scale"][0, 0])
+    assert (r["q_scale"][b, h, nqb:] == 0).all()
+    np.testing.assert_array_equal(r["k_mean"][b, h].cpu().numpy(), o["k_mean"][0, 0])
+    np.testing.assert_array_equal(r["k_scale"][b, h, :nkb].cpu().numpy(), o["k_scale"][0, 0])
+    assert (r["k_scale"][b, h, nkb:] == 0).all()
+    gv = v_e4m3[b, h].cpu().numpy()          # [N_pad, d]
+    np.testing.assert_array_equal(gv[:N], o["v_e4m3"][0, 0])
+    assert (gv[N:] == 0).all()
+    np.testing.assert_array_equal(v_scale[b, h].cpu().numpy(), o["v_scale"][0, 0])
 
 
 # --------------------------------------------------------------------------- S tiles
@@ -172,6 +177,81 @@ def test_the_largest_head_count(B, H, N, d):
     _check_quant(w, hs)
     heads = [divmod(x, H) for x in hs]
     _check_attn(w, heads=heads, nrows=None)
+
+
+def _wide_inputs(B, H, N, d, layout, P=61, seed=1777):
+    """B*H distinct heads without drawing them all on the host: P heads from
+    the seeded generator (bias and outlier channels as in the workloads), and
+    head x = b*H + h is base head x mod P with its tokens rotated by
+    (7919 x) mod N, so that neighbouring heads, and heads 2^31 elements
+    apart, hold different rows.  The device tensors are assembled from the
+    base heads by an index gather (data movement only).  Returns the device
+    q, k, v views in the layout and head(x) -> its (q, k, v) as CPU bf16
+    [1,1,N,d], rebuilt from the same base heads."""
+    bq, bk, bv, _ = make_qkv(tiny_custom(1, P, N, d, seed=seed, bias_sigma=2.0, outlier_frac=0.02))
+    BH = B * H
+
+    def head(x):
+        p, r = x % P, (7919 * x) % N
+        return tuple(t[0, p].roll(-r, dims=0).contiguous().view(1, 1, N, d) for t in (bq, bk, bv))
+
+    x = torch.arange(BH, device=DEV)
+    rows = (torch.arange(N, device=DEV).view(1, N) + ((7919 * x) % N).view(BH, 1)) % N
+    pidx = (x % P).view(BH, 1)
+    if layout == "fused":
+        buf = torch.empty(B, N, 3, H, d, dtype=torch.bfloat16, device=DEV)
+        views = tuple(buf[:, :, i].permute(0, 2, 1, 3) for i in range(3))
+    else:
+        views = tuple(torch.empty(B, H, N, d, dtype=torch.bfloat16, device=DEV) for _ in range(3))
+    for t, dst in zip((bq, bk, bv), views):
+        dst.copy_(t[0].to(DEV)[pidx, rows].view(B, H, N, d))
+    return views, head
+
+
+@pytest.mark.parametrize("layout", ["contiguous", "fused"])
+def test_tensors_past_2_31_elements(layout):
+    """65535 heads of 300 tokens (B=3, H=21845, d=128): the inputs and the
+    output hold 2.5e9 elements and the codes 3.2e9, so element offsets pass
+    2^31 (and byte offsets of the bf16 tensors 2^32); in the fused layout a
+    token's stride alone is 8.4 M elements and rows of the first batch cross
+    2^31.  Codes and scales equal the oracle's bit for bit, the forward and
+    the K-residual forward are within the parity bar, on heads at the start,
+    astride the 2^31-byte, 2^31-code and 2^31-input-element boundaries, and
+    at the end."""
+    B, H, N, d = 3, 21845, 300, 128
+    sm_scale = 1.0 / math.sqrt(d)
+    (qd, kd, vd), head = _wide_inputs(B, H, N, d, layout)
+    assert qd.numel() > 2 ** 31 and B * H * sage.n_pad(N) * d > 2 ** 31
+    xs = [0, 1, 27962, 43690, 55924, B * H - 2, B * H - 1]
+    cpu = {x: head(x) for x in xs}
+    for x in xs:  # the device copies hold the same bits as the oracle's inputs
+        b, h = divmod(x, H)
+        for dv, cv in zip((qd, kd, vd), cpu[x]):
+            assert torch.equal(dv[b, h].cpu(), cv[0, 0])
+    r = sage.sage_quant_qk(qd, kd)
+    v_e4m3, v_scale = sage.sage_quant_v(vd)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    for x in xs:
+        b, h = divmod(x, H)
+        _assert_head_codes(r, v_e4m3, v_scale, b, h, N, oracle.quantize(*cpu[x]), f"{layout} head {x}")
+    del r, v_e4m3, v_scale
+    for kres in (False, True):
+        fwd = sage.sage_attn_fwd_kres if kres else sage.sage_attn_fwd
+        out = fwd(qd, kd, vd, sm_scale=sm_scale)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        for x in xs:
+            b, h = divmod(x, H)
+            got = U.bf16_to_f64(out[b, h])
+            _, bits = oracle.attn_quant(*cpu[x], sm_scale, k_residual=kres)
+            label = f"{layout} {'K-residual ' if kres else ''}head {x}"
+            ok, rel, mx, nstep = U.within_tol(got, oracle.bf16_bits_to_f64(bits[0, 0]), label=label)
+            assert np.isfinite(got).all()
+            assert ok, (label, rel, mx, nstep)
+        del out
+    del qd, kd, vd
+    torch.cuda.empty_cache()
 
 
 def test_batched_heads_d64():
