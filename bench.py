@@ -59,16 +59,16 @@ def _peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def _attn_traffic(workload):
-    """DRAM bytes per launch of the attention kernel, as counted by ncu on this
-    workload (profiles/k_attn_traffic.txt), or None when there is no count or
-    the kernel source changed since it was taken."""
+def _profile_traffic(record, source, workload):
+    """DRAM bytes (read + written) per launch of a kernel, as counted by ncu on
+    this workload (the JSON record profiles/<record>), or None when there is no
+    count or the kernel's source (csrc/<source>) changed since it was taken."""
     import hashlib
     here = os.path.dirname(os.path.abspath(__file__))
     try:
-        with open(os.path.join(here, "profiles", "k_attn_traffic.txt")) as f:
+        with open(os.path.join(here, "profiles", record)) as f:
             rec = json.load(f)
-        with open(os.path.join(here, "quantized_attention_qk_b200", "csrc", "sage_attn.cu"), "rb") as f:
+        with open(os.path.join(here, "quantized_attention_qk_b200", "csrc", source), "rb") as f:
             sha = hashlib.sha256(f.read()).hexdigest()
     except (OSError, ValueError):
         return None
@@ -76,6 +76,28 @@ def _attn_traffic(workload):
     if rec.get("source_sha256") != sha or not w:
         return None
     return int(w["dram_bytes_read"]) + int(w["dram_bytes_write"])
+
+
+def _attn_traffic(workload):
+    return _profile_traffic("k_attn_traffic.txt", "sage_attn.cu", workload)
+
+
+# The quantize pass's algorithmic bytes per element of B*H*N*d: Q read (2) and
+# coded (1); K and V each read for their statistics (2), read again (2) and
+# coded (1).
+QPASS_BYTES_PER_ELEMENT = 13
+
+
+def _quant_roofline(w, quant_ms, hbm_gbs, peak_kind, traffic):
+    """The quantize pass against HBM bandwidth: algorithmic bytes per second
+    over the measured copy bandwidth.  quant_ms runs from the step's start
+    event to the event recorded before the attention kernel."""
+    nbytes = QPASS_BYTES_PER_ELEMENT * w.B * w.H * w.N * w.d
+    achieved = nbytes / (quant_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "kernel": "k_qpass (statistics, then codes)", "achieved": round(achieved, 1),
+            "peak": float(hbm_gbs), "unit": "GB/s", "frac": round(achieved / float(hbm_gbs), 4),
+            "traffic": traffic, "algorithmic_bytes": nbytes, "quant_ms": round(quant_ms, 4),
+            "peak_source": f"{peak_kind}: STREAM-style copy bandwidth"}
 
 
 EX2_PER_SCORE = 0.75     # the softmax takes 2^x on the MUFU unit for 6 of every 8 scores, by polynomial for 2
@@ -371,6 +393,9 @@ def run_gpu(args):
         attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
         total_ms = max_over_ranks(sum(step_ms))
         attn_avg = max_over_ranks(sum(attn_ms) / steps)
+        # the kernels before the attention kernel: the quantize pass (and, when
+        # selecting, the block selection)
+        quant_avg = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / steps)
         kept = 1.0
         if sparse:  # fraction of (query tile, key tile) pairs the selection kept, outside the timed region
             _, mask = sage.sage_attn_fwd_sparse(q, k, v, tau=args.tau, sm_scale=w.sm_scale, out=out, workspace=ws,
@@ -399,7 +424,8 @@ def run_gpu(args):
         d2h = out_host.numel() * out_host.element_size()
         del q, k, v, bufs, out, ws, host_in, ws_host
         torch.cuda.empty_cache()
-        return dict(total_ms=total_ms, attn_ms=attn_avg, e2e_ms=e2e_ms, clocks=clocks, h2d=h2d, d2h=d2h, kept=kept)
+        return dict(total_ms=total_ms, attn_ms=attn_avg, quant_ms=quant_avg, e2e_ms=e2e_ms, clocks=clocks, h2d=h2d,
+                    d2h=d2h, kept=kept)
 
     wp = WORKLOADS[args.workload]
     r = measure(wp, args.steps, args.warmup)
@@ -428,6 +454,12 @@ def run_gpu(args):
                      "peak_source": f"{peak_kind}: {PEAK_NOTE}",
                      "attn_ms": round(r["attn_ms"], 4)},
         "roofline_softmax": softmax_roofline(wp, r),
+        # the quantize pass of the dense forward (a selecting forward runs its
+        # selection before the attention kernel too; the other modes code
+        # different tensors)
+        "roofline_quantize": (_quant_roofline(wp, r["quant_ms"], peaks["hbm_gbs"], peak_kind,
+                                              _profile_traffic("k_qpass_traffic.txt", "sage_quant.cu", wp.name))
+                              if dense else None),
         "e2e": {"value": round(world * wp.ops / (r["e2e_ms"] * 1e-3) / 1e12, 2), "unit": "TOPS",
                 "ms_per_step": round(r["e2e_ms"], 4), "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"],
                 "api": "sage_attn_fwd_host (pinned host qkv -> device in head chunks on three streams, quantize + "
@@ -462,6 +494,8 @@ def run_gpu(args):
                 "attn_tops": round(attn_tops2, 2), "attn_ms": round(r2["attn_ms"], 4),
                 "attn_frac": round(attn_tops2 / peak_8bit, 4),
                 "softmax_frac": softmax_roofline(ws_, r2)["frac"],
+                "quant_ms": round(r2["quant_ms"], 4),
+                "quant_frac": _quant_roofline(ws_, r2["quant_ms"], peaks["hbm_gbs"], peak_kind, None)["frac"],
                 "e2e_tops": round(world * ws_.ops / (r2["e2e_ms"] * 1e-3) / 1e12, 2), "clocks": r2["clocks"]})
             line["gpu_launches"] += LAUNCHES_PER_STEP * k2
     if rank == 0 and world == 1 and args.cpu_baseline:

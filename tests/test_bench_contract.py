@@ -54,3 +54,32 @@ def test_softmax_roofline_takes_the_lower_ceiling():
     # a kept fraction (block-sparse) scales the scores the kernel computed
     r3 = bench._softmax_roofline(w, 0.2, 0.5, 4.0e12, 2000.0, 148, None)
     assert abs(r3["achieved"] - r2["achieved"] / 2) < 1e-4
+
+
+def test_quantize_roofline_counts_the_algorithmic_bytes():
+    """The quantize pass against HBM: 13 bytes per element of B*H*N*d (Q read
+    and coded, K and V read twice and coded) per second, over the copy
+    bandwidth."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from quantized_attention_qk_b200.inputs import WORKLOADS
+
+    w = WORKLOADS["video"]
+    r = bench._quant_roofline(w, 0.5, 6000.0, "measured", 123)
+    nbytes = 13 * w.B * w.H * w.N * w.d
+    assert r["algorithmic_bytes"] == nbytes and r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - nbytes / 0.5e-3 / 1e9) < 0.1
+    assert abs(r["frac"] - r["achieved"] / 6000.0) < 1e-4
+    assert r["traffic"] == 123 and r["quant_ms"] == 0.5
+
+
+def test_traffic_records_hold_only_for_the_source_they_were_taken_on():
+    """A DRAM count is reported only while the kernel's source has the hash the
+    record was taken on, and only for a workload it was taken on."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    for rec, src in (("k_attn_traffic.txt", "sage_attn.cu"), ("k_qpass_traffic.txt", "sage_quant.cu")):
+        assert bench._profile_traffic(rec, src, "no such workload") is None
+        assert bench._profile_traffic(rec, "sage_api.cu", "flux") is None  # another file's hash
+    assert bench._profile_traffic("no_such_record.txt", "sage_quant.cu", "flux") is None
