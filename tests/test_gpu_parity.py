@@ -290,6 +290,74 @@ def test_zero_query_gives_mean_of_quantized_v():
     assert (out[0, 0] == out[0, 0, :1]).all()
 
 
+def _one_head_against_oracle(q, k, v, sm_scale, label):
+    """The forward on one [1,1,N,d] head against the oracle's quant emulation
+    on all rows; returns (GPU output, oracle output) as float64 [N,d]."""
+    out = sage.sage_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), sm_scale=sm_scale)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    got = U.bf16_to_f64(out[0, 0])
+    _, bits = oracle.attn_quant(q, k, v, sm_scale)
+    want = oracle.bf16_bits_to_f64(bits[0, 0])
+    ok, rel, mx, nstep = U.within_tol(got, want, label=label)
+    assert np.isfinite(got).all()
+    assert ok, (label, rel, mx, nstep)
+    return got, want
+
+
+def test_scores_far_below_the_row_max_get_no_weight():
+    """Hard attention: channel 0 of the keys is +1 or -1 at random and the
+    queries point along it, so half of the keys score about 140 (in log2
+    units) below the others.  Their exponent offsets fall far below the range
+    where the FMA-pipe exponential clamps its input (and the MUFU flushes to
+    zero), in both kinds of lanes: they must get no weight, and every row is
+    a weighted mean of the top keys' V rows, as in the oracle."""
+    N, d = 1000, 128
+    g = torch.Generator().manual_seed(21)
+    top = torch.rand(N, generator=g) < 0.5
+    q = 0.05 * torch.randn(1, 1, N, d, generator=g)
+    q[..., 0] = 4.0
+    k = 0.05 * torch.randn(1, 1, N, d, generator=g)
+    k[0, 0, :, 0] = torch.where(top, 1.0, -1.0)
+    v = torch.randn(1, 1, N, d, generator=g)
+    q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+    got, want = _one_head_against_oracle(q, k, v, 12.0, "scores far below the max")
+    # the bottom keys carry nothing: the oracle's rows lie in the span of the
+    # top keys' values (their mean, within the spread of the top weights)
+    vt = U.bf16_to_f64(v[0, 0])[top.numpy()]
+    assert np.abs(want - vt.mean(axis=0)).max() < 0.25
+
+
+def test_identical_keys_give_uniform_weights():
+    """Every key the same row: the smoothed keys are exactly zero, so are the K
+    codes and scales, every score is 0 and every row is the mean of the
+    quantized V rows."""
+    N, d = 700, 64
+    g = torch.Generator().manual_seed(22)
+    q = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    k = (3.0 * torch.randn(1, 1, 1, d, generator=g)).expand(1, 1, N, d).contiguous().to(torch.bfloat16)
+    v = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    got, _ = _one_head_against_oracle(q, k, v, 1 / math.sqrt(d), "identical keys")
+    assert (got == got[:1]).all()
+
+
+def test_zero_values_give_a_zero_output():
+    N, d = 333, 128
+    g = torch.Generator().manual_seed(23)
+    q = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    k = torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16)
+    v = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    got, want = _one_head_against_oracle(q, k, v, 1 / math.sqrt(d), "zero values")
+    assert (got == 0).all() and (want == 0).all()
+
+
+def test_a_tiny_softmax_scale_gives_near_uniform_weights():
+    N, d = 500, 128
+    g = torch.Generator().manual_seed(24)
+    q, k, v = (torch.randn(1, 1, N, d, generator=g).to(torch.bfloat16) for _ in range(3))
+    _one_head_against_oracle(q, k, v, 1e-6, "tiny softmax scale")
+
+
 def test_attention_kernel_on_oracle_codes():
     """Feed the oracle's own codes and scales to the attention kernel alone: this
     isolates the tcgen05 attention from the quantize pass."""
