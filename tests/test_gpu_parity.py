@@ -290,14 +290,16 @@ def test_zero_query_gives_mean_of_quantized_v():
     assert (out[0, 0] == out[0, 0, :1]).all()
 
 
-def _one_head_against_oracle(q, k, v, sm_scale, label):
-    """The forward on one [1,1,N,d] head against the oracle's quant emulation
-    on all rows; returns (GPU output, oracle output) as float64 [N,d]."""
-    out = sage.sage_attn_fwd(q.to(DEV), k.to(DEV), v.to(DEV), sm_scale=sm_scale)
+def _one_head_against_oracle(q, k, v, sm_scale, label, kres=False):
+    """The forward (or the K-residual forward) on one [1,1,N,d] head against
+    the oracle's quant emulation on all rows; returns (GPU output, oracle
+    output) as float64 [N,d]."""
+    fwd = sage.sage_attn_fwd_kres if kres else sage.sage_attn_fwd
+    out = fwd(q.to(DEV), k.to(DEV), v.to(DEV), sm_scale=sm_scale)
     torch.cuda.synchronize()
     sage.sage_check()
     got = U.bf16_to_f64(out[0, 0])
-    _, bits = oracle.attn_quant(q, k, v, sm_scale)
+    _, bits = oracle.attn_quant(q, k, v, sm_scale, k_residual=kres)
     want = oracle.bf16_bits_to_f64(bits[0, 0])
     ok, rel, mx, nstep = U.within_tol(got, want, label=label)
     assert np.isfinite(got).all()
@@ -305,13 +307,15 @@ def _one_head_against_oracle(q, k, v, sm_scale, label):
     return got, want
 
 
-def test_scores_far_below_the_row_max_get_no_weight():
+@pytest.mark.parametrize("kres", [False, True], ids=["smoothing", "k_residual"])
+def test_scores_far_below_the_row_max_get_no_weight(kres):
     """Hard attention: channel 0 of the keys is +1 or -1 at random and the
     queries point along it, so half of the keys score about 140 (in log2
     units) below the others.  Their exponent offsets fall far below the range
     where the FMA-pipe exponential clamps its input (and the MUFU flushes to
     zero), in both kinds of lanes: they must get no weight, and every row is
-    a weighted mean of the top keys' V rows, as in the oracle."""
+    a weighted mean of the top keys' V rows, as in the oracle (also with
+    K-residual quantization, where the block means carry much of the score)."""
     N, d = 1000, 128
     g = torch.Generator().manual_seed(21)
     top = torch.rand(N, generator=g) < 0.5
@@ -321,7 +325,7 @@ def test_scores_far_below_the_row_max_get_no_weight():
     k[0, 0, :, 0] = torch.where(top, 1.0, -1.0)
     v = torch.randn(1, 1, N, d, generator=g)
     q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
-    got, want = _one_head_against_oracle(q, k, v, 12.0, "scores far below the max")
+    got, want = _one_head_against_oracle(q, k, v, 12.0, "scores far below the max", kres=kres)
     # the bottom keys carry nothing: the oracle's rows lie in the span of the
     # top keys' values (their mean, within the spread of the top weights)
     vt = U.bf16_to_f64(v[0, 0])[top.numpy()]

@@ -164,6 +164,40 @@ def test_selection_matches_the_oracle(w):
     assert torch.equal(used, again)
 
 
+def test_tied_tile_scores_keep_the_lowest_key_tiles():
+    """Every key the same row: the smoothed K codes are all zero, so every
+    tile score ties at 0 and the ranking falls back to the key tile's index
+    (reading S3: lower index first).  Each query tile keeps the shortest
+    prefix of key tiles whose token count reaches tau of N (the last tile is
+    ragged), the same mask as the oracle's, and the forward with it equals
+    the oracle's masked emulation."""
+    B, H, N, d = 1, 2, 1100, 128
+    g = torch.Generator().manual_seed(541)
+    q = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    k = (2.0 * torch.randn(B, H, 1, d, generator=g)).expand(B, H, N, d).contiguous().to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    sm_scale = d ** -0.5
+    nt = -(-N // T)
+    sizes = np.minimum(T, N - T * np.arange(nt))
+    sbar_o = oracle.block_scores(q, k, v, sm_scale)
+    assert (sbar_o == 0).all()
+    dev = tuple(t.to(DEV) for t in (q, k, v))
+    codes = sage.sage_quant_qk(dev[0], dev[1])
+    for tau in (0.05, 0.5, 0.93, 1.0):
+        keep_o = oracle.block_select(sbar_o, N, tau).astype(bool)
+        n_keep = int(np.searchsorted(np.cumsum(sizes), tau * N - 1e-9) + 1)  # shortest prefix reaching tau*N
+        assert (keep_o == (np.arange(nt) < min(n_keep, nt))).all(), tau
+        mask = sage.sage_block_select(codes, N, sm_scale, tau)
+        out, used = sage.sage_attn_fwd_sparse(*dev, tau=tau, sm_scale=sm_scale, return_mask=True)
+        torch.cuda.synchronize()
+        sage.sage_check()
+        assert np.array_equal(sage.mask_to_keep(mask, nt).cpu().numpy(), keep_o), tau
+        assert torch.equal(used, mask)
+        _, bits = oracle.attn_quant(q, k, v, sm_scale, kv_keep=keep_o.astype(np.uint8))
+        ok, rel, mx, nstep = U.within_tol(U.bf16_to_f64(out), oracle.bf16_bits_to_f64(bits), label=f"ties tau {tau}")
+        assert ok, (tau, rel, mx, nstep)
+
+
 def test_tau_forward_matches_the_oracle():
     """The selecting forward against the oracle's selection and masked
     emulation: the same kept sets on every row, outputs within the
