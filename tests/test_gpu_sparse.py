@@ -198,6 +198,45 @@ def test_tied_tile_scores_keep_the_lowest_key_tiles():
         assert ok, (tau, rel, mx, nstep)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_the_largest_tile_count(d):
+    """N = 4096 * 128 tokens: the most key tiles one selection ranks (4096,
+    in shared memory), and at d = 128 the attention kernel's largest shared
+    memory (its step lists for 4096 query tiles on top of the tiles).  The
+    tile scores and the kept sets equal the oracle's bit for bit on every
+    query tile, the selecting forward uses that mask, and its sampled rows
+    are within the bar.  The keys carry an offset that falls along the
+    sequence, so every row of scores is sorted up to local disorder (which
+    keeps the oracle's insertion-sort ranking quick)."""
+    B, H, N = 1, 1, 4096 * T
+    nt = N // T
+    g = torch.Generator().manual_seed(561)
+    u = torch.randn(d, generator=g)
+    u = u / u.norm() * 4.0
+    fall = torch.linspace(1.0, -1.0, nt).repeat_interleave(T).view(1, 1, N, 1)
+    q = (0.5 * torch.randn(B, H, N, d, generator=g) + u).to(torch.bfloat16)
+    k = (0.5 * torch.randn(B, H, N, d, generator=g) + fall * u).to(torch.bfloat16)
+    v = torch.randn(B, H, N, d, generator=g).to(torch.bfloat16)
+    sm_scale, tau = d ** -0.5, 0.3
+    sbar_o = oracle.block_scores(q, k, v, sm_scale)
+    keep_o = oracle.block_select(sbar_o, N, tau)
+    assert 0.02 < keep_o.mean() < 0.5
+    dev = tuple(t.to(DEV) for t in (q, k, v))
+    codes = sage.sage_quant_qk(dev[0], dev[1])
+    mask, sbar_g = sage.sage_block_select(codes, N, sm_scale, tau, want_scores=True)
+    out, used = sage.sage_attn_fwd_sparse(*dev, tau=tau, sm_scale=sm_scale, return_mask=True)
+    torch.cuda.synchronize()
+    sage.sage_check()
+    np.testing.assert_array_equal(sbar_g.cpu().numpy(), sbar_o)
+    assert np.array_equal(sage.mask_to_keep(mask, nt).cpu().numpy(), keep_o.astype(bool))
+    assert torch.equal(used, mask)
+    rows = U.sample_rows(N, 24, seed=5)
+    _, bits = oracle.attn_quant(q, k, v, sm_scale, rows=rows, kv_keep=keep_o)
+    got = U.bf16_to_f64(out[0, 0, torch.from_numpy(rows).long().to(DEV)])
+    ok, rel, mx, nstep = U.within_tol(got, oracle.bf16_bits_to_f64(bits[0, 0]), label="4096 tiles")
+    assert ok, (rel, mx, nstep)
+
+
 def test_tau_forward_matches_the_oracle():
     """The selecting forward against the oracle's selection and masked
     emulation: the same kept sets on every row, outputs within the
