@@ -35,11 +35,12 @@
  *     (b, h, n, c) order; the channel stride must be 1.  A fused [B,N,3,H,d]
  *     qkv buffer is passed as three views with strides (N*3*H*d, d, 3*H*d, 1)
  *     and read in place (no copy).
- *   - Inputs and output are bf16.  d must be 64 or 128; N >= 1; B, H >= 1.
- *     Base pointers must be 16-byte aligned and the b, h, n strides multiples
- *     of 8 elements (16-byte vectors).  Otherwise SAGE_ERR_INVALID_ARG (bad
- *     pointer/stride/shape/scale) or SAGE_ERR_UNSUPPORTED (d, dtype) is
- *     returned before anything is launched.
+ *   - Inputs and output are bf16.  d must be 64 or 128; N >= 1; B, H >= 1;
+ *     B*H <= 65535 and N <= 2^24.  Base pointers must be 16-byte aligned and
+ *     the b, h, n strides multiples of 8 elements (16-byte vectors).
+ *     Otherwise SAGE_ERR_INVALID_ARG (bad pointer/stride/shape/scale) or
+ *     SAGE_ERR_UNSUPPORTED (d, B*H, N) is returned before anything is
+ *     launched, and every size query below answers 0 for such a shape.
  *   - Input values are finite.  With an infinity or NaN in a block the codes of
  *     that block (and every output that uses them) are unspecified; nothing
  *     checks for it.
@@ -245,8 +246,8 @@ size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d);
  * Enqueued after the work already on `stream`; `stream` continues after the
  * whole call (out_host is complete once `stream` reaches that point).
  * Errors: SAGE_ERR_INVALID_ARG (null buffer, layout, shape, sm_scale),
- * SAGE_ERR_UNSUPPORTED (d), SAGE_ERR_WORKSPACE (scratch too small),
- * SAGE_ERR_CUDA.  The pages have no counterpart; this is the call a serving
+ * SAGE_ERR_UNSUPPORTED (d; B*H > 65535 or N > 2^24, the limits of every
+ * entry point), SAGE_ERR_WORKSPACE (scratch too small), SAGE_ERR_CUDA.  The pages have no counterpart; this is the call a serving
  * path with host-resident tensors makes.
  */
 sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_host,

@@ -87,12 +87,19 @@ sage_status_t get_scratch(Scratch &s, void *ws, size_t ws_bytes, size_t need, cu
 
 }  // namespace
 
+constexpr int64_t kMaxHeads = 65535;   // B*H: the attention grid's second dimension
+constexpr int kMaxTokens = 1 << 24;
+
 sage_status_t check_shape(int B, int H, int N, int d) {
     if (B < 1 || H < 1 || N < 1) return fail(SAGE_ERR_INVALID_ARG, "shape B=%d H=%d N=%d must be positive", B, H, N);
     if (d != 64 && d != 128) return fail(SAGE_ERR_UNSUPPORTED, "head dim d=%d is not supported (64 or 128)", d);
-    if ((int64_t)B * H > 65535) return fail(SAGE_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
-    if (N > (1 << 24)) return fail(SAGE_ERR_UNSUPPORTED, "N=%d exceeds 2^24 tokens", N);
+    if ((int64_t)B * H > kMaxHeads) return fail(SAGE_ERR_UNSUPPORTED, "B*H=%lld exceeds 65535", (long long)B * H);
+    if (N > kMaxTokens) return fail(SAGE_ERR_UNSUPPORTED, "N=%d exceeds 2^24 tokens", N);
     return SAGE_OK;
+}
+
+bool shape_supported(int B, int H, int N, int d) {
+    return B >= 1 && H >= 1 && N >= 1 && (d == 64 || d == 128) && (int64_t)B * H <= kMaxHeads && N <= kMaxTokens;
 }
 
 sage_status_t check_on_current_device(const void *p, const char *name) {
@@ -191,12 +198,12 @@ sage_status_t sage_check(sage_stream_t stream) {
 }
 
 size_t sage_quant_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     return stats_ws_bytes(Shape{B, H, N, d});
 }
 
 size_t sage_attn_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     const Shape s{B, H, N, d};
     return up(codes_bytes(s)) + stats_ws_bytes(s);
 }
@@ -333,14 +340,14 @@ static sage_status_t check_tau(float tau) {
 }
 
 size_t sage_block_mask_bytes(int B, int H, int N) {
-    if (B < 1 || H < 1 || N < 1) return 0;
+    if (!shape_supported(B, H, N, 128)) return 0;
     const Shape s{B, H, N, 128};
     if (s.n_tiles() > kMaxSelectTiles) return 0;
     return mask_bytes(s);
 }
 
 size_t sage_block_select_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     const Shape s{B, H, N, d};
     if (s.n_tiles() > kMaxSelectTiles) return 0;
     return select_ws_bytes(s);
@@ -366,7 +373,7 @@ sage_status_t sage_block_select(const int8_t *q_i8, const float *q_scale, const 
 }
 
 size_t sage_attn_sparse_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     const Shape s{B, H, N, d};
     if (s.n_tiles() > kMaxSelectTiles) return 0;
     return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + up(select_ws_bytes(s)) + up(mask_bytes(s));
@@ -458,7 +465,7 @@ static size_t kres_bmean_bytes(const Shape &s) { return up((size_t)s.BH() * s.n_
 static size_t kres_slot_bytes(const Shape &s) { return up((size_t)kres_slots() * s.n_kblocks() * 256 * 4); }
 
 size_t sage_attn_kres_workspace_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     const Shape s{B, H, N, d};
     if (kres_slots() <= 0) return 0;
     return up(codes_bytes(s)) + up(stats_ws_bytes(s)) + kres_bmean_bytes(s) + kres_slot_bytes(s);

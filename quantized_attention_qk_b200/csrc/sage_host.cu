@@ -81,7 +81,7 @@ using namespace sage;
 extern "C" {
 
 size_t sage_attn_fwd_host_scratch_bytes(int B, int H, int N, int d) {
-    if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+    if (!shape_supported(B, H, N, d)) return 0;
     const size_t elems = (size_t)B * H * N * d;
     return up(3 * elems * 2) + up(elems * 2) + kStreams * chunk_ws_bytes(chunk_heads(B, H, N, d), N, d);
 }
@@ -96,14 +96,7 @@ sage_status_t sage_attn_fwd_host(const void *qkv_host, int layout, void *out_hos
         set_last_error("layout %d is neither SAGE_LAYOUT_FUSED nor SAGE_LAYOUT_CONTIGUOUS", layout);
         return SAGE_ERR_INVALID_ARG;
     }
-    if (B < 1 || H < 1 || N < 1) {
-        set_last_error("shape B=%d H=%d N=%d must be positive", B, H, N);
-        return SAGE_ERR_INVALID_ARG;
-    }
-    if (d != 64 && d != 128) {
-        set_last_error("head dim d=%d is not supported (64 or 128)", d);
-        return SAGE_ERR_UNSUPPORTED;
-    }
+    if (sage_status_t r = check_shape(B, H, N, d)) return r;
     if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) {
         set_last_error("sm_scale must be finite and positive");
         return SAGE_ERR_INVALID_ARG;

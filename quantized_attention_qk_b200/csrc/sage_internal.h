@@ -76,6 +76,9 @@ void set_last_error(const char *fmt, ...);
 // current device (kernels launch on the current device; a pointer of another
 // device would be read across the interconnect or fault).
 sage_status_t check_shape(int B, int H, int N, int d);
+// The shapes check_shape accepts, without recording an error (for the size
+// queries, which answer 0 for every other shape).
+bool shape_supported(int B, int H, int N, int d);
 sage_status_t check_on_current_device(const void *p, const char *name);
 
 size_t stats_ws_bytes(const Shape &s);

@@ -52,6 +52,16 @@ def test_workspace_sizes(L):
         assert sage.sage_quant_workspace_bytes(B, H, N, d) > 0
     assert sage.sage_attn_workspace_bytes(1, 1, 128, 96) == 0
     assert sage.sage_attn_workspace_bytes(1, 1, 0, 64) == 0
+    # every size query answers 0 for the shapes the calls reject (B*H past
+    # 65535, N past 2^24), and no size arithmetic runs for them
+    for fn in (sage.sage_attn_workspace_bytes, sage.sage_quant_workspace_bytes,
+               sage.sage_attn_sparse_workspace_bytes, sage.sage_attn_fwd_host_scratch_bytes):
+        assert fn(2, 32768, 128, 64) == 0 and fn(1, 1, (1 << 24) + 1, 64) == 0
+        assert fn(65535, 1, 128, 64) > 0 and fn(1, 65535, 128, 64) > 0
+        assert fn(46341, 46341, 128, 64) == 0      # B*H past 2^31 too
+    L.sage_block_select_workspace_bytes.restype = ctypes.c_size_t
+    assert L.sage_block_select_workspace_bytes(2, 32768, 128, 64) == 0
+    assert sage.sage_block_mask_bytes(2, 32768, 128) == 0 and sage.sage_block_mask_bytes(1, 65535, 128) > 0
 
 
 def _call_fwd(L, q=16 * 4096, strides=(8 * 4096, 4096 * 8, 8 * 8, 1), B=1, H=1, N=128, d=64, scale=0.125):
@@ -97,11 +107,16 @@ def test_host_forward_rejects_bad_arguments_before_any_launch(L):
     assert f(p, 2, p, 1, 1, 8, 64, 0.125, None, 0, None) == 1             # unknown layout
     assert f(p, 0, p, 1, 1, 8, 96, 0.125, None, 0, None) == 2             # head dim
     assert f(p, 1, p, 1, 0, 8, 64, 0.125, None, 0, None) == 1             # shape
+    assert f(p, 1, p, 2, 32768, 8, 64, 0.125, None, 0, None) == 2         # B*H past 65535
+    assert f(p, 1, p, 1, 1, (1 << 24) + 1, 64, 0.125, None, 0, None) == 2  # N past 2^24
     assert f(p, 1, p, 1, 1, 8, 64, float("nan"), None, 0, None) == 1      # sm_scale
     assert f(p, 1, p, 1, 1, 8, 64, 0.125, p, 16, None) == 3               # scratch too small
     L.sage_attn_fwd_host_scratch_bytes.restype = ctypes.c_size_t
     assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 128) > 3 * 24 * 4608 * 128 * 2 + 24 * 4608 * 128 * 2
     assert L.sage_attn_fwd_host_scratch_bytes(1, 24, 4608, 96) == 0
+    assert L.sage_attn_fwd_host_scratch_bytes(2, 32768, 8, 64) == 0
+    assert L.sage_attn_fwd_host_scratch_bytes(1, 1, (1 << 24) + 1, 64) == 0
+    assert L.sage_attn_fwd_host_scratch_bytes(1, 65535, 8, 64) > 0
 
 
 def _call_sparse(L, tau=0.5, N=128, d=64, mask_in=None, mask_out=None, q=16 * 4096):
